@@ -1,0 +1,20 @@
+"""B200 (sm_100a) forward pass of jagged, target-aware HSTU pointwise (SiLU) attention.
+
+    out = Mask(SiLU(alpha * Q K^T)) V / N
+
+over jagged batches of user-interaction histories with appended candidate tokens (history
+causal, each candidate sees all history plus itself), plus the streaming variant that queries
+only new tokens against a cached K/V prefix.  The work happens in ``libhstu_attn.so`` (C ABI in
+``include/hstu_attn.h``); :mod:`.binding` marshals torch tensors into it.  The binding's names
+are re-exported lazily so that :mod:`.workloads` and :mod:`.metrics` import without it.
+"""
+_BINDING_NAMES = ("HstuError", "hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_get_error",
+                  "hstu_attn_schedule", "hstu_attn_schedule_capacity", "hstu_attn_status_string",
+                  "library_path", "load_library")
+
+
+def __getattr__(name):
+    if name in _BINDING_NAMES:
+        from . import binding
+        return getattr(binding, name)
+    raise AttributeError(name)

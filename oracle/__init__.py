@@ -1,0 +1,146 @@
+"""fp64 CPU oracle for jagged target-aware HSTU pointwise (SiLU) attention.
+
+TEST INFRASTRUCTURE ONLY.  The oracle is a plain, slow, obviously-correct restatement of what
+the CUDA library computes; it exists to check that library and shares no code with it.  Only
+``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline / reference leg may
+import it.  The library never falls back to it.
+
+Computation (pages: the DLRMv3 MLPerf review, section "model selection" — attention is
+Mask(SiLU(Q K^T)) V without relative bias, the history encoding is shared by all candidates
+and its K/V reused across timestamps; the infolabhq.com multi-stage page — the user side never
+depends on a candidate, and target-aware attention weighs history against each candidate):
+
+    out[i,h,:] = (1/N) * sum_{j in A(i)} silu(alpha * q[i,h,:].k[j,h,:]) * v[j,h,:]
+    A(i) = {j <= i} for a history token (i < U); {j < U} + {i} for a candidate (i >= U)
+
+The C source (``hstu_oracle.c``) holds the arithmetic; this module only marshals numpy arrays.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+class Oracle:
+    """ctypes view of one build of the C oracle (the default build, or a test's mutant build)."""
+
+    def __init__(self, path):
+        lib = ctypes.CDLL(path)
+        f32p = ctypes.POINTER(ctypes.c_float)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        f64p = ctypes.POINTER(ctypes.c_double)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+        lib.hstu_oracle_fwd.argtypes = [f32p, f32p, f32p, i32p, i32p, i32, i32, i32, i64, f64,
+                                        f64, f64p, i64p]
+        lib.hstu_oracle_fwd_cached.argtypes = [f32p, f32p, f32p, i32p, i32p, i32p, i32, i32, i32,
+                                               i64, i64, f64, f64, f64p, i64p]
+        lib.hstu_oracle_rows.argtypes = [f32p, f32p, f32p, i32p, i32p, i32p, i32, i32, i32, i64,
+                                         i64, f64, f64, i32p, i32p, i64, f64p, i64p]
+        for fn in (lib.hstu_oracle_fwd, lib.hstu_oracle_fwd_cached, lib.hstu_oracle_rows,
+                   lib.hstu_oracle_num_threads):
+            fn.restype = ctypes.c_int
+        self.lib = lib
+
+    def num_threads(self) -> int:
+        """Threads the oracle's OpenMP loops use (OMP_NUM_THREADS or all cores)."""
+        return int(self.lib.hstu_oracle_num_threads())
+
+    def fwd(self, q, k, v, seq_offsets, num_targets, alpha, N, return_macs=False):
+        """Full forward: q, k, v [total, H, d]; returns float64 [total, H, d]."""
+        q, k, v = _f32(q), _f32(k), _f32(v)
+        off = _i32(seq_offsets)
+        nt = None if num_targets is None else _i32(num_targets)
+        total, H, d = q.shape
+        out = np.zeros((total, H, d), dtype=np.float64)
+        macs = ctypes.c_int64(0)
+        rc = self.lib.hstu_oracle_fwd(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                      _ptr(v, ctypes.c_float), _ptr(off, ctypes.c_int32),
+                                      _ptr(nt, ctypes.c_int32), len(off) - 1, H, d, total,
+                                      float(alpha), float(N), _ptr(out, ctypes.c_double),
+                                      ctypes.byref(macs))
+        if rc != 0:
+            raise ValueError("oracle: inconsistent seq_offsets / num_targets")
+        return (out, macs.value) if return_macs else out
+
+    def fwd_cached(self, q_new, k, v, seq_offsets, num_targets, cached_len, alpha, N,
+                   return_macs=False):
+        """Streaming forward: q_new [total_q, H, d] new rows; k, v [total_kv, H, d] full segments."""
+        q_new, k, v = _f32(q_new), _f32(k), _f32(v)
+        off = _i32(seq_offsets)
+        nt = None if num_targets is None else _i32(num_targets)
+        cl = None if cached_len is None else _i32(cached_len)
+        total_q, H, d = q_new.shape
+        out = np.zeros((total_q, H, d), dtype=np.float64)
+        macs = ctypes.c_int64(0)
+        rc = self.lib.hstu_oracle_fwd_cached(_ptr(q_new, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                             _ptr(v, ctypes.c_float), _ptr(off, ctypes.c_int32),
+                                             _ptr(nt, ctypes.c_int32), _ptr(cl, ctypes.c_int32),
+                                             len(off) - 1, H, d, k.shape[0], total_q, float(alpha),
+                                             float(N), _ptr(out, ctypes.c_double), ctypes.byref(macs))
+        if rc != 0:
+            raise ValueError("oracle: inconsistent seq_offsets / num_targets / cached_len")
+        return (out, macs.value) if return_macs else out
+
+    def rows(self, q, k, v, seq_offsets, num_targets, cached_len, alpha, N, row_user, row_local,
+             return_macs=False):
+        """Selected output rows [n, H, d] for (user, local query row) pairs; cached_len may be None."""
+        q, k, v = _f32(q), _f32(k), _f32(v)
+        off = _i32(seq_offsets)
+        nt = None if num_targets is None else _i32(num_targets)
+        cl = None if cached_len is None else _i32(cached_len)
+        ru, rl = _i32(row_user), _i32(row_local)
+        total_q, H, d = q.shape
+        out = np.zeros((len(ru), H, d), dtype=np.float64)
+        macs = ctypes.c_int64(0)
+        rc = self.lib.hstu_oracle_rows(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                       _ptr(v, ctypes.c_float), _ptr(off, ctypes.c_int32),
+                                       _ptr(nt, ctypes.c_int32), _ptr(cl, ctypes.c_int32),
+                                       len(off) - 1, H, d, k.shape[0], total_q, float(alpha),
+                                       float(N), _ptr(ru, ctypes.c_int32), _ptr(rl, ctypes.c_int32),
+                                       len(ru), _ptr(out, ctypes.c_double), ctypes.byref(macs))
+        if rc != 0:
+            raise ValueError("oracle: inconsistent offsets or row selection")
+        return (out, macs.value) if return_macs else out
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _i32(a):
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def _ptr(a, ctype):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+_default = None
+
+
+def default() -> Oracle:
+    """The oracle built from oracle/hstu_oracle.c (compiled on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle(_build.build())
+    return _default
+
+
+def num_threads() -> int:
+    return default().num_threads()
+
+
+def fwd(*args, **kwargs):
+    return default().fwd(*args, **kwargs)
+
+
+def fwd_cached(*args, **kwargs):
+    return default().fwd_cached(*args, **kwargs)
+
+
+def rows(*args, **kwargs):
+    return default().rows(*args, **kwargs)
