@@ -1,0 +1,402 @@
+"""Benchmark of jagged target-aware HSTU pointwise (SiLU) attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one forward pass of the attention (work plan + attention kernel) over one batch of
+the DLRMv3-shaped workload: 8 users x (2048 history + 2048 candidate tokens), H=4 heads of
+d=128, bf16 N(0,1)/sqrt(d) inputs, alpha=1/sqrt(128), N=4096 (synthetic: the DLRMv3 dataset is
+not available).  Inputs are resident in HBM; L2 is flushed (256 MiB write) before every timed
+step.  Multi-GPU: one process per GPU, each with its own batch (users are independent, so the
+batch is sharded by user with no collective on the data path; weak scaling); the only
+collectives are the barrier and the max-over-ranks of the device time.
+
+Prints one JSON line on rank 0.  `value` is whole-job algorithmic TFLOP/s (visible query/key
+pairs only, both matmuls); `e2e` is the same metric through the one-shot public entry point
+with host buffers and the host<->device copies inside the timed region; `roofline` reports the
+attention kernel against the measured dense-bf16 tensor peak; `cpu_baseline` times the fp64
+oracle on the host cores on a bounded sample of the same workload.
+
+`--impl reference`: this method has no published implementation; the reference arm is the fp64
+oracle on the host cores (rank 0 only), each step a bounded sample of the same workload.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "jagged SiLU-attention TFLOP/s & target tokens/s, % of B200 BF16 TC peak"
+WORKLOAD = "dlrmv3"
+FALLBACK_PEAK_TFLOPS = 1590.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------------------------ ranks
+class Ranks:
+    """RANK / WORLD_SIZE from the launcher; a process group only when there is more than one."""
+
+    def __init__(self, backend="nccl"):
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float, device=None) -> float:
+        if self.pg is None:
+            return float(x)
+        import torch
+        t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, x: float, device=None) -> float:
+        if self.pg is None:
+            return float(x)
+        import torch
+        t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch of the same shape."""
+    return base_seed + 1000 * rank
+
+
+# ------------------------------------------------------------------------------------ clocks
+_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read only) while the timed loop runs."""
+
+    def __init__(self, device_index, interval_s=0.02):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = int(pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM))
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self.interval = interval_s
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(int(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)))
+                bits = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+                for b, name in _REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------ helpers
+def measured_peak():
+    """Dense bf16 tensor peak in TFLOP/s: the measured burst figure if present, else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "measured burst (MEASURED_PEAKS.json bf16_tflops)"
+    except Exception:
+        return FALLBACK_PEAK_TFLOPS, "fallback 1.59 PFLOP/s"
+
+
+def workload_config(w, n_gpus):
+    return {
+        "workload": "%s: %d users x (%d history + %d candidates), H=%d, d=%d, alpha=1/sqrt(%d), N=%d" % (
+            w.name, w.B, int(w.uih_len[0]), int(w.num_targets[0]), w.H, w.d, w.d, int(w.N)),
+        "users_per_gpu": w.B,
+        "global_batch": w.B * n_gpus,
+        "seq_len": int(w.seq_len.max()),
+        "heads": w.H,
+        "head_dim": w.d,
+        "parallelism": "dp%d (users sharded, no collective)" % n_gpus,
+        "l2": "flushed before every timed step (256 MiB write)",
+    }
+
+
+def oracle_sample_rows(w, n_rows, seed):
+    """A stratified sample of query rows (history and candidates in proportion) of the workload."""
+    rng = np.random.default_rng(seed)
+    users = rng.integers(0, w.B, size=n_rows)
+    L = w.seq_len[users]
+    local = (rng.random(n_rows) * L).astype(np.int64)
+    return users.astype(np.int32), local.astype(np.int32)
+
+
+def time_oracle(w, n_rows, seed):
+    """Runs the oracle on a row sample; returns (seconds, algorithmic flops of the sample)."""
+    import oracle
+    users, local = oracle_sample_rows(w, n_rows, seed)
+    t0 = time.perf_counter()
+    _, macs = oracle.rows(w.q, w.k, w.v, w.seq_offsets, w.num_targets, None, w.alpha, w.N, users, local,
+                          return_macs=True)
+    dt = time.perf_counter() - t0
+    return dt, 2 * macs
+
+
+# ------------------------------------------------------------------------------------ arms
+def run_ours(args, ranks):
+    import torch
+    from hstu_pointwise_attention_jagged_b200 import binding, metrics, workloads
+
+    dev = torch.device("cuda", ranks.local_rank)
+    torch.cuda.set_device(dev)
+    binding.load_library()
+    w = workloads.make(WORKLOAD, seed=rank_seed(1, ranks.rank))
+    flops = metrics.algorithmic_flops(w.seq_offsets, w.num_targets, w.H, w.d)
+    targets = int(w.num_targets.sum())
+
+    def to_bf16(x):
+        return torch.from_numpy(workloads.bf16_bits(x).view(np.int16)).view(torch.bfloat16)
+
+    q_h, k_h, v_h = (to_bf16(x).pin_memory() for x in (w.q, w.k, w.v))
+    off_h = torch.from_numpy(w.seq_offsets.astype(np.int32)).pin_memory()
+    nt_h = torch.from_numpy(w.num_targets.astype(np.int32)).pin_memory()
+    q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
+    off, nt = off_h.to(dev), nt_h.to(dev)
+    out = torch.empty_like(q)
+    plan = torch.empty((binding.hstu_attn_plan_bytes(w.B, w.H, w.total),), dtype=torch.uint8, device=dev)
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    msl = w.max_seq_len
+
+    def step():
+        binding.hstu_attn_plan(off, nt, None, w.H, w.total, w.total, msl, plan=plan, stream=stream)
+
+    def attn():
+        binding.hstu_attn_fwd_planned(q, k, v, off, nt, None, w.alpha, w.N, plan, out=out, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+        attn()
+    torch.cuda.synchronize()
+    status = binding.hstu_attn_get_error()
+    if status != 0:
+        raise RuntimeError("warm-up reported %s" % binding.hstu_attn_status_string(status))
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    ranks.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+            attn()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        ranks.barrier()
+    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
+    attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    status = binding.hstu_attn_get_error()
+    if status != 0:
+        raise RuntimeError("timed steps reported %s" % binding.hstu_attn_status_string(status))
+    total_ms = ranks.max(sum(step_ms), dev)
+    attn_total_ms = ranks.max(sum(attn_ms), dev)
+    ms_per_step = total_ms / K
+    job_flops = ranks.sum(flops, dev)
+    job_targets = ranks.sum(targets, dev)
+    value = job_flops / (ms_per_step * 1e-3) / 1e12
+    attn_avg_ms = attn_total_ms / K
+    achieved = flops / (attn_avg_ms * 1e-3) / 1e12
+    peak, peak_src = measured_peak()
+
+    # End to end: the one-shot public call with host buffers, copies inside the timed region.
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    E = max(3, min(args.steps, 50))
+    h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h, off_h, nt_h))
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        off.copy_(off_h, non_blocking=True)
+        nt.copy_(nt_h, non_blocking=True)
+        binding.hstu_attn_fwd(q, k, v, off, nt, w.alpha, w.N, msl, out=out, stream=stream)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ranks.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    e2e_ms = ranks.max(e0.elapsed_time(e1), dev) / E
+    e2e_value = job_flops / (e2e_ms * 1e-3) / 1e12
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": ranks.world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt(d) bf16; DLRMv3 dataset unavailable)",
+        "config": workload_config(w, ranks.world),
+        "target_tokens_per_s": round(job_targets / (ms_per_step * 1e-3), 1),
+        "pct_of_peak": round(100.0 * value / ranks.world / peak, 2),
+        "algorithmic_gflop_per_step": round(job_flops / 1e9, 3),
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "api": "hstu_attn_fwd (plan + attention) with pinned host buffers"},
+        "gpu_launches": 2 * K,
+        "roofline": {"bound": "tensor", "kernel": "hstu_fwd_kernel<128>", "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": args.traffic, "peak_source": peak_src,
+                     "attn_ms_per_launch": round(attn_avg_ms, 5),
+                     "flops_per_launch": int(flops)},
+        "clocks": sampler.summary(),
+    }
+    if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline:
+        import oracle
+        cores = oracle.num_threads()
+        t0 = time.perf_counter()
+        _, macs = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N, return_macs=True)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": 2 * macs / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": "one full step: every row and head of the same batch (fp64 C oracle, "
+                                          "OpenMP), %.1f s" % dt}
+    return line
+
+
+def run_reference(args, world):
+    """The fp64 oracle on the host cores, rank 0 only: each step a bounded row sample, sized so that
+    warm-up plus K steps stay near a minute of CPU work."""
+    import oracle
+    from hstu_pointwise_attention_jagged_b200 import workloads
+    w = workloads.make(WORKLOAD, seed=rank_seed(1, 0))
+    cores = oracle.num_threads()
+    rows = args.ref_rows or int(min(8000, max(16, 240000 // (args.steps + args.warmup))))
+    for i in range(args.warmup):
+        time_oracle(w, rows, seed=900 + i)
+    secs, fl = 0.0, 0
+    for i in range(args.steps):
+        dt, f = time_oracle(w, rows, seed=1000 + i)
+        secs += dt
+        fl += f
+    value = fl / secs / 1e12
+    ms_step = secs / args.steps * 1e3
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0,1)/sqrt(d) bf16 values; DLRMv3 dataset unavailable)",
+        "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": "each step: %d random query rows x %d heads of the batch" % (rows, w.H)},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--ref-rows", type=int, default=0, help="rows per step of the reference arm (0: sized from K)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per attention launch from an ncu capture of this kernel, if current")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        ap.error("--gpus %d but WORLD_SIZE=%d (launch N>1 with torch.distributed.run)" % (args.gpus, world))
+    if args.impl == "reference":
+        # Rank 0 alone runs the CPU oracle; other ranks exit without work (no process group).
+        if int(os.environ.get("RANK", "0")) == 0:
+            print(json.dumps(run_reference(args, world)), flush=True)
+        return 0
+    ranks = Ranks(backend="nccl")
+    try:
+        line = run_ours(args, ranks)
+    finally:
+        ranks.close()
+    if ranks.rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,228 @@
+"""ctypes binding of libhstu_attn.so (C ABI: include/hstu_attn.h).
+
+Argument marshalling only: every function checks the torch tensors it is given, passes their
+device pointers, sizes and the current CUDA stream to the C entry point of the same name, and
+raises :class:`HstuError` on a non-zero status.  All arithmetic happens in the library's CUDA
+kernels; there is no other code path.  If the library has not been built the first call raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libhstu_attn.so")
+_lib = None
+
+STATUS = {
+    0: "HSTU_OK",
+    1: "HSTU_ERR_INVALID_ARGUMENT",
+    2: "HSTU_ERR_UNSUPPORTED",
+    3: "HSTU_ERR_CUDA",
+    4: "HSTU_ERR_BAD_OFFSETS",
+    5: "HSTU_ERR_TIMEOUT",
+}
+
+# Every symbol include/hstu_attn.h declares.
+EXPORTS = (
+    "hstu_attn_fwd",
+    "hstu_attn_fwd_cached",
+    "hstu_attn_plan_bytes",
+    "hstu_attn_plan",
+    "hstu_attn_fwd_planned",
+    "hstu_attn_get_error",
+    "hstu_attn_status_string",
+)
+
+
+class HstuError(RuntimeError):
+    """A libhstu_attn call returned a status other than HSTU_OK."""
+
+    def __init__(self, status, where):
+        self.status = int(status)
+        super().__init__("%s: %s" % (where, STATUS.get(self.status, "status %d" % self.status)))
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Loads libhstu_attn.so once; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError("libhstu_attn.so is not built (run __graft_entry__.build() or "
+                           "python -m hstu_pointwise_attention_jagged_b200.build)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    lib.hstu_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp]
+    lib.hstu_attn_fwd_cached.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, f32,
+                                         vp, vp]
+    i64 = ctypes.c_int64
+    lib.hstu_attn_plan_bytes.argtypes = [i32, i32, i32]
+    lib.hstu_attn_plan_bytes.restype = i64
+    lib.hstu_attn_plan.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, i64, vp]
+    lib.hstu_attn_fwd_planned.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp]
+    lib.hstu_attn_get_error.argtypes = [vp]
+    lib.hstu_attn_status_string.argtypes = [ctypes.c_int]
+    lib.hstu_attn_status_string.restype = ctypes.c_char_p
+    for name in ("hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_plan", "hstu_attn_fwd_planned",
+                 "hstu_attn_get_error"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _stream_ptr(stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_tokens(name, t, H=None, d=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != torch.bfloat16 or t.dim() != 3 or not t.is_contiguous():
+        raise TypeError("%s must be a contiguous bf16 tensor [rows, H, d]" % name)
+    if H is not None and (t.shape[1] != H or t.shape[2] != d):
+        raise ValueError("%s has shape %s, expected [*, %d, %d]" % (name, tuple(t.shape), H, d))
+
+
+def _check_index(name, t, n, device, optional=True):
+    if t is None:
+        if optional:
+            return
+        raise TypeError("%s is required" % name)
+    if not isinstance(t, torch.Tensor) or t.device != device or t.dtype != torch.int32 or \
+            t.dim() != 1 or not t.is_contiguous() or t.numel() != n:
+        raise TypeError("%s must be a contiguous int32 tensor of %d elements on %s" % (name, n, device))
+
+
+def _raise_if(status, where):
+    if status != 0:
+        raise HstuError(status, where)
+
+
+def hstu_attn_fwd(q, k, v, seq_offsets, num_targets, alpha, N, max_seq_len, out=None, stream=None):
+    """Full forward pass; returns ``out`` (bf16 [total, H, d]). See include/hstu_attn.h."""
+    lib = load_library()
+    _check_tokens("q", q)
+    total, H, d = q.shape
+    _check_tokens("k", k, H, d)
+    _check_tokens("v", v, H, d)
+    if k.shape[0] != total or v.shape[0] != total:
+        raise ValueError("q, k and v must have the same number of rows")
+    B = seq_offsets.numel() - 1
+    _check_index("seq_offsets", seq_offsets, B + 1, q.device, optional=False)
+    _check_index("num_targets", num_targets, B, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tokens("out", out, H, d)
+    with torch.cuda.device(q.device):
+        st = lib.hstu_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(num_targets), B, H, d,
+                               total, int(max_seq_len), float(alpha), float(N), _ptr(out),
+                               _stream_ptr(stream, q.device))
+    _raise_if(st, "hstu_attn_fwd")
+    return out
+
+
+def hstu_attn_fwd_cached(q, k, v, seq_offsets, num_targets, cached_len, alpha, N, max_seq_len, out=None,
+                         stream=None):
+    """Streaming forward: new-token queries against cached prefix + new K/V; returns ``out``."""
+    lib = load_library()
+    _check_tokens("q", q)
+    total_q, H, d = q.shape
+    _check_tokens("k", k, H, d)
+    _check_tokens("v", v, H, d)
+    total_kv = k.shape[0]
+    if v.shape[0] != total_kv:
+        raise ValueError("k and v must have the same number of rows")
+    B = seq_offsets.numel() - 1
+    _check_index("seq_offsets", seq_offsets, B + 1, q.device, optional=False)
+    _check_index("num_targets", num_targets, B, q.device)
+    _check_index("cached_len", cached_len, B, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tokens("out", out, H, d)
+    with torch.cuda.device(q.device):
+        st = lib.hstu_attn_fwd_cached(_ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(num_targets),
+                                      _ptr(cached_len), B, H, d, total_kv, total_q, int(max_seq_len),
+                                      float(alpha), float(N), _ptr(out), _stream_ptr(stream, q.device))
+    _raise_if(st, "hstu_attn_fwd_cached")
+    return out
+
+
+def hstu_attn_plan_bytes(B, H, total_q):
+    """Bytes of a plan buffer for these sizes (see include/hstu_attn.h for its layout)."""
+    return int(load_library().hstu_attn_plan_bytes(int(B), int(H), int(total_q)))
+
+
+def hstu_attn_plan(seq_offsets, num_targets, cached_len, H, total_kv, total_q, max_seq_len, plan=None,
+                   stream=None):
+    """Builds the work plan on the device; returns the plan (uint8 CUDA tensor)."""
+    lib = load_library()
+    B = seq_offsets.numel() - 1
+    dev = seq_offsets.device
+    _check_index("seq_offsets", seq_offsets, B + 1, dev, optional=False)
+    _check_index("num_targets", num_targets, B, dev)
+    _check_index("cached_len", cached_len, B, dev)
+    nbytes = hstu_attn_plan_bytes(B, H, total_q)
+    if plan is None:
+        plan = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=dev)
+    if plan.dtype != torch.uint8 or not plan.is_contiguous() or plan.device != dev:
+        raise TypeError("plan must be a contiguous uint8 tensor on %s" % dev)
+    with torch.cuda.device(dev):
+        st = lib.hstu_attn_plan(_ptr(seq_offsets), _ptr(num_targets), _ptr(cached_len), B, int(H), int(total_kv),
+                                int(total_q), int(max_seq_len), _ptr(plan), plan.numel(), _stream_ptr(stream, dev))
+    _raise_if(st, "hstu_attn_plan")
+    return plan
+
+
+def hstu_attn_fwd_planned(q, k, v, seq_offsets, num_targets, cached_len, alpha, N, plan, out=None, stream=None):
+    """Attention over a plan from hstu_attn_plan (same offsets); returns ``out``."""
+    lib = load_library()
+    _check_tokens("q", q)
+    total_q, H, d = q.shape
+    _check_tokens("k", k, H, d)
+    _check_tokens("v", v, H, d)
+    total_kv = k.shape[0]
+    B = seq_offsets.numel() - 1
+    _check_index("seq_offsets", seq_offsets, B + 1, q.device, optional=False)
+    _check_index("num_targets", num_targets, B, q.device)
+    _check_index("cached_len", cached_len, B, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tokens("out", out, H, d)
+    with torch.cuda.device(q.device):
+        st = lib.hstu_attn_fwd_planned(_ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(num_targets),
+                                       _ptr(cached_len), B, H, d, total_kv, total_q, float(alpha), float(N),
+                                       _ptr(plan), _ptr(out), _stream_ptr(stream, q.device))
+    _raise_if(st, "hstu_attn_fwd_planned")
+    return out
+
+
+def plan_contents(plan, B):
+    """Reads a plan's header, query-row starts and valid items back to the host (inspection)."""
+    raw = plan.cpu().numpy().view("<i4")
+    header = raw[:4].copy()
+    qs_words = ((B * 4 + 15) // 16) * 4
+    q_start = raw[4:4 + B].copy()
+    items = raw[4 + qs_words:].reshape(-1, 4)[:int(header[1])].copy()
+    return header, q_start, items
+
+
+def hstu_attn_get_error(device=None, stream=None):
+    """Synchronises the stream and returns (and clears) the device error status (0 = clean)."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(lib.hstu_attn_get_error(_stream_ptr(stream, dev)))
+
+
+def hstu_attn_status_string(status):
+    return load_library().hstu_attn_status_string(int(status)).decode()

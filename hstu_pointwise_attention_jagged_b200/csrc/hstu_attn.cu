@@ -1,0 +1,352 @@
+// hstu_attn.cu — host side of libhstu_attn.so: the C ABI declared in include/hstu_attn.h.
+//
+// Per call: validate arguments on the host -> take a stream-ordered workspace from the
+// library's per-device memory pool -> schedule_kernel (work list from seq_offsets /
+// num_targets / cached_len) -> hstu_fwd_kernel<d> (persistent, one CTA per SM) -> return the
+// workspace on the same stream.  Nothing synchronises; nothing falls back to another path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <functional>
+#include <mutex>
+
+#include "hstu_attn.h"
+#include "hstu_fwd_sm100.cuh"
+#include "schedule.cuh"
+
+namespace hstu {
+
+// Device error word (kErrBadOffsets | kErrTimeout), one per device context.
+__device__ unsigned g_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  std::once_flag once;
+  cudaError_t init_err = cudaSuccess;
+  int num_sms = 0;
+  cudaMemPool_t pool = nullptr;
+  unsigned* err_word = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+
+std::once_flag g_encode_once;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+template <int D>
+cudaError_t set_kernel_attrs() {
+  return cudaFuncSetAttribute(hstu_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              FwdCfg<D>::kSmemBytes);
+}
+
+// One-time per-device set-up, run with that device current.
+void init_device(DeviceState& st, int dev) {
+  cudaError_t e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) {
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    e = cudaMemPoolCreate(&st.pool, &props);
+  }
+  if (e == cudaSuccess) {
+    // Keep up to 64 MiB cached between calls so steady-state calls never reach the driver.
+    uint64_t keep = 64ull << 20;
+    e = cudaMemPoolSetAttribute(st.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+  }
+  if (e == cudaSuccess) e = cudaGetSymbolAddress(reinterpret_cast<void**>(&st.err_word), g_error_word);
+  if (e == cudaSuccess) e = set_kernel_attrs<32>();
+  if (e == cudaSuccess) e = set_kernel_attrs<64>();
+  if (e == cudaSuccess) e = set_kernel_attrs<128>();
+  st.init_err = e;
+}
+
+DeviceState* device_state() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  DeviceState& st = g_dev[dev];
+  std::call_once(st.once, init_device, std::ref(st), dev);
+  return st.init_err == cudaSuccess ? &st : nullptr;
+}
+
+bool encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 2-D bf16 tensor map over a jagged [rows, H*d] matrix; box = (box_x columns, 128 rows).
+bool encode_rows(CUtensorMap* map, const void* base, int64_t rows, int64_t row_elems, uint32_t box_x,
+                 CUtensorMapSwizzle swz) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_elems), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_elems) * 2u};
+  cuuint32_t box[2] = {box_x, static_cast<cuuint32_t>(kTileRows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Plan layout (documented in include/hstu_attn.h):
+//   int32 header[4] = {work counter, num_items, done counter, 0}
+//   int32 q_start[B], padded to 16 bytes
+//   int4  items[capacity] = {b, pair, h, cost}, capacity = H * (total_q / 256 + B)
+struct Plan {
+  int32_t* counter;
+  int32_t* num_items;
+  int32_t* done;
+  int32_t* q_start;
+  int4* items;
+};
+
+int64_t capacity(int32_t B, int32_t H, int32_t total_q) {
+  return static_cast<int64_t>(H) * (total_q / kPairRows + B);
+}
+
+int64_t plan_bytes(int32_t B, int32_t H, int32_t total_q) {
+  return 16 + ((static_cast<int64_t>(B) * 4 + 15) / 16) * 16 + capacity(B, H, total_q) * 16;
+}
+
+Plan carve(void* base, int32_t B) {
+  uint8_t* p = static_cast<uint8_t*>(base);
+  Plan w;
+  w.counter = reinterpret_cast<int32_t*>(p);
+  w.num_items = reinterpret_cast<int32_t*>(p + 4);
+  w.done = reinterpret_cast<int32_t*>(p + 8);
+  w.q_start = reinterpret_cast<int32_t*>(p + 16);
+  w.items = reinterpret_cast<int4*>(p + 16 + ((static_cast<size_t>(B) * 4 + 15) / 16) * 16);
+  return w;
+}
+
+int cost_bins(int32_t max_seq_len) {
+  // A 256-row item computes at most 2 * (ceil(L/128) + 1) score tiles.
+  int64_t n = 2 * (static_cast<int64_t>(max_seq_len) / kTileRows + 3) + 1;
+  return static_cast<int>(n < kMaxCostBins ? n : kMaxCostBins);
+}
+
+// Scalar checks shared by every entry point.  Returns HSTU_OK or the status to report.
+hstu_status_t check_sizes(int32_t B, int32_t H, int32_t total_kv, int32_t total_q) {
+  if (B < 0 || H < 1 || total_kv < 0 || total_q < 0 || total_q > total_kv) return HSTU_ERR_INVALID_ARGUMENT;
+  if (capacity(B, H, total_q) > INT_MAX) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+hstu_status_t check_tokens(const void* q, const void* k, const void* v, const int32_t* seq_offsets, int32_t H,
+                           int32_t d, int32_t total_kv, int32_t total_q, float alpha, float N, const void* out) {
+  if (!std::isfinite(alpha) || !std::isfinite(N) || !(N > 0.0f)) return HSTU_ERR_INVALID_ARGUMENT;
+  if (d != 32 && d != 64 && d != 128) return HSTU_ERR_UNSUPPORTED;
+  const int64_t row_elems = static_cast<int64_t>(H) * d;
+  if (row_elems > INT_MAX / 2) return HSTU_ERR_UNSUPPORTED;
+  if (total_q == 0) return HSTU_OK;  // nothing is read or written; empty tensors may be NULL
+  if (!q || !k || !v || !seq_offsets || !out) return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return HSTU_ERR_UNSUPPORTED;
+  const size_t qbytes = static_cast<size_t>(total_q) * row_elems * 2;
+  const size_t kvbytes = static_cast<size_t>(total_kv) * row_elems * 2;
+  if (overlaps(out, qbytes, q, qbytes) || overlaps(out, qbytes, k, kvbytes) || overlaps(out, qbytes, v, kvbytes))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  return HSTU_OK;
+}
+
+cudaError_t launch_plan(const int32_t* seq_offsets, const int32_t* num_targets, const int32_t* cached_len,
+                        int32_t B, int32_t H, int32_t total_kv, int32_t total_q, int32_t max_seq_len,
+                        const Plan& w, unsigned* err, cudaStream_t stream) {
+  SchedArgs a;
+  a.seq_offsets = seq_offsets;
+  a.num_targets = num_targets;
+  a.cached_len = cached_len;
+  a.B = B;
+  a.H = H;
+  a.total_kv = total_kv;
+  a.total_q = total_q;
+  a.max_seq_len = max_seq_len;
+  a.nbins = cost_bins(max_seq_len);
+  a.max_items = static_cast<int32_t>(capacity(B, H, total_q));
+  a.q_start = w.q_start;
+  a.items = w.items;
+  a.num_items = w.num_items;
+  a.work_counter = w.counter;
+  a.done_counter = w.done;
+  a.err = err;
+  schedule_kernel<<<1, kSchedThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                       int grid, cudaStream_t stream) {
+  hstu_fwd_kernel<D><<<grid, kNumThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+// The attention kernel over a plan built for the same offsets.  Arguments already checked.
+hstu_status_t launch_attention(DeviceState* st, const void* q, const void* k, const void* v,
+                               const int32_t* seq_offsets, const int32_t* num_targets, const int32_t* cached_len,
+                               int32_t B, int32_t H, int32_t d, int32_t total_kv, int32_t total_q, float alpha,
+                               float N, void* plan, void* out, cudaStream_t stream) {
+  if (!encoder()) return HSTU_ERR_CUDA;
+  const int64_t row_elems = static_cast<int64_t>(H) * d;
+  CUtensorMap tq, tk, tv;
+  const uint32_t box_x = d >= 64 ? 64u : 32u;
+  const CUtensorMapSwizzle swz = d >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!encode_rows(&tq, q, total_q, row_elems, box_x, swz) || !encode_rows(&tk, k, total_kv, row_elems, box_x, swz) ||
+      !encode_rows(&tv, v, total_kv, row_elems, box_x, swz))
+    return HSTU_ERR_CUDA;
+  const Plan w = carve(plan, B);
+  FwdParams p;
+  p.seq_offsets = seq_offsets;
+  p.num_targets = num_targets;
+  p.cached_len = cached_len;
+  p.q_start = w.q_start;
+  p.items = w.items;
+  p.num_items = w.num_items;
+  p.work_counter = w.counter;
+  p.done_counter = w.done;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.H = H;
+  p.half_alpha = 0.5f * alpha;
+  p.inv_n = 1.0f / N;
+  p.err = st->err_word;
+  const int64_t cap = capacity(B, H, total_q);
+  const int grid = static_cast<int>(cap < st->num_sms ? cap : st->num_sms);
+  cudaError_t e;
+  if (d == 128) e = launch_fwd<128>(tq, tk, tv, p, grid, stream);
+  else if (d == 64) e = launch_fwd<64>(tq, tk, tv, p, grid, stream);
+  else e = launch_fwd<32>(tq, tk, tv, p, grid, stream);
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// Plan into a stream-ordered buffer from the library's pool, attention, return the buffer.
+hstu_status_t run(const void* q, const void* k, const void* v, const int32_t* seq_offsets,
+                  const int32_t* num_targets, const int32_t* cached_len, int32_t B, int32_t H, int32_t d,
+                  int32_t total_kv, int32_t total_q, int32_t max_seq_len, float alpha, float N, void* out,
+                  void* stream_ptr) {
+  hstu_status_t s = check_sizes(B, H, total_kv, total_q);
+  if (s == HSTU_OK && max_seq_len < 0) s = HSTU_ERR_INVALID_ARGUMENT;
+  if (s == HSTU_OK) s = check_tokens(q, k, v, seq_offsets, H, d, total_kv, total_q, alpha, N, out);
+  if (s != HSTU_OK) return s;
+  if (B == 0 || total_q == 0) return HSTU_OK;
+  DeviceState* st = device_state();
+  if (!st) return HSTU_ERR_CUDA;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  void* plan = nullptr;
+  if (cudaMallocFromPoolAsync(&plan, static_cast<size_t>(plan_bytes(B, H, total_q)), st->pool, stream) !=
+      cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (launch_plan(seq_offsets, num_targets, cached_len, B, H, total_kv, total_q, max_seq_len, carve(plan, B),
+                  st->err_word, stream) != cudaSuccess)
+    s = HSTU_ERR_CUDA;
+  if (s == HSTU_OK)
+    s = launch_attention(st, q, k, v, seq_offsets, num_targets, cached_len, B, H, d, total_kv, total_q, alpha, N,
+                         plan, out, stream);
+  if (cudaFreeAsync(plan, stream) != cudaSuccess && s == HSTU_OK) s = HSTU_ERR_CUDA;
+  return s;
+}
+
+}  // namespace
+}  // namespace hstu
+
+extern "C" {
+
+hstu_status_t hstu_attn_fwd(const void* q, const void* k, const void* v, const int32_t* seq_offsets,
+                            const int32_t* num_targets, int32_t B, int32_t H, int32_t d, int32_t total_tokens,
+                            int32_t max_seq_len, float alpha, float N, void* out, void* stream) {
+  return hstu::run(q, k, v, seq_offsets, num_targets, nullptr, B, H, d, total_tokens, total_tokens, max_seq_len,
+                   alpha, N, out, stream);
+}
+
+hstu_status_t hstu_attn_fwd_cached(const void* q, const void* k, const void* v, const int32_t* seq_offsets,
+                                   const int32_t* num_targets, const int32_t* cached_len, int32_t B, int32_t H,
+                                   int32_t d, int32_t total_kv, int32_t total_q, int32_t max_seq_len, float alpha,
+                                   float N, void* out, void* stream) {
+  return hstu::run(q, k, v, seq_offsets, num_targets, cached_len, B, H, d, total_kv, total_q, max_seq_len, alpha,
+                   N, out, stream);
+}
+
+int64_t hstu_attn_plan_bytes(int32_t B, int32_t H, int32_t total_q) {
+  if (B < 0 || H < 1 || total_q < 0) return 0;
+  return hstu::plan_bytes(B, H, total_q);
+}
+
+hstu_status_t hstu_attn_plan(const int32_t* seq_offsets, const int32_t* num_targets, const int32_t* cached_len,
+                             int32_t B, int32_t H, int32_t total_kv, int32_t total_q, int32_t max_seq_len,
+                             void* plan, int64_t plan_bytes, void* stream_ptr) {
+  hstu_status_t s = hstu::check_sizes(B, H, total_kv, total_q);
+  if (s != HSTU_OK) return s;
+  if (max_seq_len < 0 || !plan || plan_bytes < hstu::plan_bytes(B, H, total_q)) return HSTU_ERR_INVALID_ARGUMENT;
+  if (B > 0 && !seq_offsets) return HSTU_ERR_INVALID_ARGUMENT;
+  if (!hstu::aligned16(plan)) return HSTU_ERR_UNSUPPORTED;
+  hstu::DeviceState* st = hstu::device_state();
+  if (!st) return HSTU_ERR_CUDA;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  if (B == 0) return cudaMemsetAsync(plan, 0, 16, stream) == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  return hstu::launch_plan(seq_offsets, num_targets, cached_len, B, H, total_kv, total_q, max_seq_len,
+                           hstu::carve(plan, B), st->err_word, stream) == cudaSuccess
+             ? HSTU_OK
+             : HSTU_ERR_CUDA;
+}
+
+hstu_status_t hstu_attn_fwd_planned(const void* q, const void* k, const void* v, const int32_t* seq_offsets,
+                                    const int32_t* num_targets, const int32_t* cached_len, int32_t B, int32_t H,
+                                    int32_t d, int32_t total_kv, int32_t total_q, float alpha, float N,
+                                    void* plan, void* out, void* stream_ptr) {
+  hstu_status_t s = hstu::check_sizes(B, H, total_kv, total_q);
+  if (s == HSTU_OK) s = hstu::check_tokens(q, k, v, seq_offsets, H, d, total_kv, total_q, alpha, N, out);
+  if (s != HSTU_OK) return s;
+  if (B == 0 || total_q == 0) return HSTU_OK;
+  if (!plan) return HSTU_ERR_INVALID_ARGUMENT;
+  if (!hstu::aligned16(plan)) return HSTU_ERR_UNSUPPORTED;
+  hstu::DeviceState* st = hstu::device_state();
+  if (!st) return HSTU_ERR_CUDA;
+  return hstu::launch_attention(st, q, k, v, seq_offsets, num_targets, cached_len, B, H, d, total_kv, total_q,
+                                alpha, N, plan, out, static_cast<cudaStream_t>(stream_ptr));
+}
+
+hstu_status_t hstu_attn_get_error(void* stream_ptr) {
+  hstu::DeviceState* st = hstu::device_state();
+  if (!st) return HSTU_ERR_CUDA;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  unsigned word = 0;
+  if (cudaMemcpyAsync(&word, st->err_word, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (cudaMemsetAsync(st->err_word, 0, sizeof(unsigned), stream) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (word & hstu::kErrTimeout) return HSTU_ERR_TIMEOUT;
+  if (word & hstu::kErrBadOffsets) return HSTU_ERR_BAD_OFFSETS;
+  return HSTU_OK;
+}
+
+const char* hstu_attn_status_string(hstu_status_t s) {
+  switch (s) {
+    case HSTU_OK: return "HSTU_OK";
+    case HSTU_ERR_INVALID_ARGUMENT: return "HSTU_ERR_INVALID_ARGUMENT";
+    case HSTU_ERR_UNSUPPORTED: return "HSTU_ERR_UNSUPPORTED";
+    case HSTU_ERR_CUDA: return "HSTU_ERR_CUDA";
+    case HSTU_ERR_BAD_OFFSETS: return "HSTU_ERR_BAD_OFFSETS";
+    case HSTU_ERR_TIMEOUT: return "HSTU_ERR_TIMEOUT";
+  }
+  return "HSTU_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,225 @@
+// schedule.cuh — tile geometry of the target-aware mask and the device-side work-list builder.
+//
+// Mask (DLRMv3 review, section "model selection": history encoded once and shared by every
+// candidate; infolabhq.com multi-stage page: the user side never depends on a candidate, and
+// target-aware attention weighs the history against each candidate):
+//   query at position i of a segment with U history tokens may see key j iff
+//     i <  U : j <= i                 (history token, causal over the history)
+//     i >= U : j <  U  or  j == i     (candidate: all history, then itself)
+// The keys visible to a block of queries at positions [p0, p1) are therefore
+//     [0, p1)                         if p1 <= U
+//     [0, U)  +  [max(p0, U), p1)     otherwise,
+// i.e. at most two runs of 128-key tiles.  Tiles outside them are never enumerated.
+#pragma once
+
+#include <cstdint>
+
+namespace hstu {
+
+constexpr int kTileRows = 128;  // query rows per half / keys per key tile
+constexpr int kPairRows = 256;  // query rows per work item (two 128-row halves)
+
+__host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// Key tiles [0, e1) followed by [s2, e2), with s2 >= e1 (an empty second run has s2 == e2).
+struct TileRange {
+  int e1, s2, e2;
+};
+
+__host__ __device__ __forceinline__ TileRange key_tiles(int p0, int p1, int U) {
+  TileRange r{0, 0, 0};
+  if (p1 <= p0) return r;
+  if (p1 <= U) {
+    r.e1 = cdiv(p1, kTileRows);
+    r.s2 = r.e2 = r.e1;
+    return r;
+  }
+  r.e1 = cdiv(U, kTileRows);
+  const int s = (p0 > U ? p0 : U) / kTileRows;
+  const int e = cdiv(p1, kTileRows);
+  if (s <= r.e1) {
+    r.e1 = (e > r.e1) ? e : r.e1;
+    r.s2 = r.e2 = r.e1;
+  } else {
+    r.s2 = s;
+    r.e2 = e;
+  }
+  return r;
+}
+
+__host__ __device__ __forceinline__ int tile_count(const TileRange& r) { return r.e1 + (r.e2 - r.s2); }
+__host__ __device__ __forceinline__ int tile_at(const TileRange& r, int idx) {
+  return idx < r.e1 ? idx : r.s2 + (idx - r.e1);
+}
+__host__ __device__ __forceinline__ bool tile_in(const TileRange& r, int t) {
+  return t < r.e1 || (t >= r.s2 && t < r.e2);
+}
+
+// Score tiles computed by one work item: query rows [256*pair, 256*pair + nrows) at positions
+// pos0.. of a segment with U history tokens, split into two 128-row halves.
+__host__ __device__ __forceinline__ int pair_cost(int pos0, int nrows, int U) {
+  int c = 0;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int lo = hh * kTileRows;
+    const int hi = (nrows < lo + kTileRows) ? nrows : lo + kTileRows;
+    if (hi > lo) c += tile_count(key_tiles(pos0 + lo, pos0 + hi, U));
+  }
+  return c;
+}
+
+constexpr unsigned kErrBadOffsets = 1u;
+constexpr unsigned kErrTimeout = 2u;
+
+constexpr int kSchedThreads = 1024;
+constexpr int kMaxCostBins = 4096;
+
+struct SchedArgs {
+  const int32_t* seq_offsets;  // [B+1]
+  const int32_t* num_targets;  // [B] or null
+  const int32_t* cached_len;   // [B] or null
+  int32_t B, H, total_kv, total_q, max_seq_len, nbins, max_items;
+  int32_t* q_start;       // [B] out: first query row of each user, -1 if the user is skipped
+  int4* items;            // [max_items] out: {b, pair, h, cost}, non-increasing cost
+  int32_t* num_items;     // [1] out
+  int32_t* work_counter;  // [1] out: reset to 0 for the attention kernel's dynamic scheduler
+  int32_t* done_counter;  // [1] out: reset to 0 (CTAs of the attention kernel that finished)
+  unsigned* err;          // device error word
+};
+
+// Inclusive block-wide prefix sum of one value per thread (kSchedThreads threads); also
+// returns the block total.  `scratch` holds 32 ints.
+__device__ __forceinline__ long long block_inclusive_scan(long long v, long long* scratch,
+                                                          long long* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    long long n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) scratch[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = scratch[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      long long n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    scratch[lane] = w;
+  }
+  __syncthreads();
+  if (warp > 0) v += scratch[warp - 1];
+  *total = scratch[31];
+  __syncthreads();
+  return v;
+}
+
+// One CTA of kSchedThreads threads.  Validates every user, assigns query-row starts, and writes
+// the work items sorted by non-increasing cost (counting sort over cost bins; ties in any order).
+__global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs a) {
+  __shared__ int hist[kMaxCostBins];
+  __shared__ long long scan_scratch[32];
+  __shared__ long long carry_s;
+  const int tid = threadIdx.x;
+  const int nbins = a.nbins;
+
+  for (int i = tid; i < nbins; i += kSchedThreads) hist[i] = 0;
+  if (tid == 0) {
+    carry_s = 0;
+    if (a.seq_offsets[0] != 0 || a.seq_offsets[a.B] != a.total_kv) atomicOr(a.err, kErrBadOffsets);
+  }
+  __syncthreads();
+
+  // Pass 1: per-user validation, query-row starts (exclusive prefix sum of new rows), cost
+  // histogram.
+  for (int base = 0; base < a.B; base += kSchedThreads) {
+    const int b = base + tid;
+    long long nq = 0;  // query rows this user occupies in the caller's q / out layout
+    bool ok = false;
+    int L = 0, T = 0, c = 0;
+    if (b < a.B) {
+      const int o0 = a.seq_offsets[b], o1 = a.seq_offsets[b + 1];
+      L = o1 - o0;
+      T = a.num_targets ? a.num_targets[b] : 0;
+      c = a.cached_len ? a.cached_len[b] : 0;
+      ok = o0 >= 0 && L >= 0 && o1 <= a.total_kv && L <= a.max_seq_len && T >= 0 && T <= L &&
+           c >= 0 && c <= L - T;
+      if (!ok) atomicOr(a.err, kErrBadOffsets);
+      // A skipped user still owns its rows of the layout, so later users keep their places.
+      const int cc = c < 0 ? 0 : c;
+      nq = L > cc ? (long long)(L - cc) : 0;
+    }
+    long long tot;
+    const long long incl = block_inclusive_scan(nq, scan_scratch, &tot);
+    const long long start = carry_s + incl - nq;
+    if (b < a.B) {
+      if (ok && start + nq > a.total_q) {
+        ok = false;
+        atomicOr(a.err, kErrBadOffsets);
+      }
+      a.q_start[b] = ok ? (int)start : -1;
+      if (ok) {
+        const int U = L - T;
+        const int npairs = cdiv(L - c, kPairRows);
+        for (int p = 0; p < npairs; ++p) {
+          const int rows = (L - c) - p * kPairRows;
+          int cost = pair_cost(c + p * kPairRows, rows < kPairRows ? rows : kPairRows, U);
+          cost = cost < nbins ? cost : nbins - 1;
+          atomicAdd(&hist[cost], a.H);
+        }
+      }
+    }
+    __syncthreads();
+    if (tid == 0) carry_s += tot;
+    __syncthreads();
+  }
+  if (tid == 0 && carry_s != a.total_q) atomicOr(a.err, kErrBadOffsets);
+
+  // Pass 2: bin start = number of items in strictly costlier bins (descending order).
+  const int per = cdiv(nbins, kSchedThreads);
+  long long part = 0;
+  for (int k = 0; k < per; ++k) {
+    const int bin = nbins - 1 - (tid * per + k);
+    if (bin >= 0) part += hist[bin];
+  }
+  __syncthreads();
+  long long tot;
+  const long long incl = block_inclusive_scan(part, scan_scratch, &tot);
+  long long run = incl - part;
+  for (int k = 0; k < per; ++k) {
+    const int bin = nbins - 1 - (tid * per + k);
+    if (bin >= 0) {
+      const int n = hist[bin];
+      hist[bin] = (int)run;
+      run += n;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    *a.num_items = (int)(tot < a.max_items ? tot : a.max_items);
+    *a.work_counter = 0;
+    *a.done_counter = 0;
+  }
+
+  // Pass 3: scatter items into their bins.
+  for (int b = tid; b < a.B; b += kSchedThreads) {
+    const int qs = a.q_start[b];
+    if (qs < 0) continue;
+    const int L = a.seq_offsets[b + 1] - a.seq_offsets[b];
+    const int T = a.num_targets ? a.num_targets[b] : 0;
+    const int c = a.cached_len ? a.cached_len[b] : 0;
+    const int U = L - T;
+    const int npairs = cdiv(L - c, kPairRows);
+    for (int p = 0; p < npairs; ++p) {
+      const int rows = (L - c) - p * kPairRows;
+      const int cost = pair_cost(c + p * kPairRows, rows < kPairRows ? rows : kPairRows, U);
+      const int bin = cost < nbins ? cost : nbins - 1;
+      const int pos = atomicAdd(&hist[bin], a.H);
+      for (int h = 0; h < a.H; ++h)
+        if (pos + h < a.max_items) a.items[pos + h] = make_int4(b, p, h, cost);
+    }
+  }
+}
+
+}  // namespace hstu

@@ -1,0 +1,183 @@
+/*
+ * hstu_attn.h — C ABI of libhstu_attn.so: forward pass of jagged, target-aware
+ * HSTU pointwise (SiLU) attention on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (per user b, head h, query position i of user b's segment):
+ *
+ *     out[i,h,:] = (1/N) * sum_{j in A(i)} silu(alpha * <q[i,h,:], k[j,h,:]>) * v[j,h,:]
+ *
+ *     silu(x) = x / (1 + exp(-x))
+ *     A(i)    = { j : j <= i }            if i <  U_b   (history token: causal over history)
+ *             = { j : j <  U_b } + { i }  if i >= U_b   (candidate: all history, then itself)
+ *
+ * Sources (page title, then section):
+ *   - "DLRMv3: MLPerf Inference generative recommendation benchmark" (winzheng.jp review),
+ *     section "model selection", time/position-encoding paragraph: DLRMv3 drops the
+ *     relative bias, so attention is Mask(SiLU(Q K^T)) V.
+ *   - same page, same section, FLOP-formula paragraph: one history (UIH) encoding is shared
+ *     by all ~2K candidates of a request, and UIH-related K/V state is reused across a
+ *     user's consecutive timestamps (the cached variant below).
+ *   - infolabhq.com "multi-stage sequence model" page, section on the offline user model:
+ *     the user-side representation never depends on an ad candidate (history tokens never
+ *     see candidates); section "Target-Aware Multi-Head Attention": every layer re-weights
+ *     past actions against the candidate being scored (candidates see all history).
+ *   - voagi.com DLRM/TorchRec tutorial, section 2.1: jagged data = concatenated values plus
+ *     a lengths vector; a zero length is legal.  Here seq_offsets is the exclusive prefix
+ *     sum of the lengths.
+ *   The scale alpha and the normaliser 1/N are not printed on the pages; they are explicit
+ *   scalar arguments (one value per call).
+ *
+ * Layout.  All token tensors are jagged [total, H, d] bf16, row-major, heads interleaved:
+ * element (t, h, c) sits at ((size_t)t * H + h) * d + c.  User b owns rows
+ * [seq_offsets[b], seq_offsets[b+1]).  Its last num_targets[b] rows are the candidates
+ * (targets); the first U_b = L_b - T_b rows are its history.
+ *
+ * Ownership.  The caller owns every buffer.  Pointers must stay valid until the work
+ * queued on `stream` has completed; the library keeps none of them after it returns.
+ * hstu_attn_fwd / hstu_attn_fwd_cached take a small stream-ordered plan buffer (work list,
+ * work counter) from the library's own per-device memory pool and return it on the same
+ * stream; hstu_attn_plan / hstu_attn_fwd_planned use a plan buffer the caller owns.
+ * When total_q (or total_tokens) is 0 nothing is read or written and the token pointers may
+ * be NULL.
+ *
+ * Errors.  Bad scalars or NULL pointers return HSTU_ERR_INVALID_ARGUMENT synchronously and
+ * launch nothing; an unsupported head size or a misaligned pointer returns
+ * HSTU_ERR_UNSUPPORTED; a failed launch returns HSTU_ERR_CUDA.  Problems that only the
+ * device can see (inconsistent seq_offsets / num_targets / cached_len, a pipeline wait
+ * that ran past its time limit) are recorded in a per-device error word and reported by
+ * hstu_attn_get_error().  Users whose offsets are inconsistent are skipped (their output
+ * rows are not written).  Nothing in the library traps or aborts.
+ *
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ * Every call is asynchronous on that stream; calls are re-entrant and thread-safe.
+ *
+ * Inputs must be finite: rows past a user's end that share a tile with its last rows are
+ * read (and masked to an exact zero weight), so a NaN/Inf in a neighbouring user's V row
+ * could leak through 0 * Inf.
+ */
+#ifndef HSTU_ATTN_H_
+#define HSTU_ATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum hstu_status {
+  HSTU_OK = 0,
+  HSTU_ERR_INVALID_ARGUMENT = 1, /* NULL pointer, negative size, N <= 0, non-finite alpha/N */
+  HSTU_ERR_UNSUPPORTED = 2,      /* d not in {32, 64, 128}, H*d*2 not a multiple of 16 bytes, misaligned base */
+  HSTU_ERR_CUDA = 3,             /* a CUDA runtime/driver call failed */
+  HSTU_ERR_BAD_OFFSETS = 4,      /* device-detected: offsets not monotone / out of range, T_b > L_b, cached_len_b > U_b */
+  HSTU_ERR_TIMEOUT = 5           /* device-detected: a pipeline wait exceeded its time limit */
+} hstu_status_t;
+
+/*
+ * hstu_attn_fwd — full forward pass over a jagged batch.
+ *
+ *   q, k, v       device, bf16 [total_tokens, H, d], 16-byte aligned base addresses.
+ *   seq_offsets   device, int32 [B+1]: seq_offsets[0] = 0, non-decreasing,
+ *                 seq_offsets[B] = total_tokens.  L_b = seq_offsets[b+1] - seq_offsets[b].
+ *   num_targets   device, int32 [B], 0 <= T_b <= L_b; NULL means every T_b = 0 (plain causal).
+ *   B             number of users (>= 0; B = 0 or total_tokens = 0 launches nothing).
+ *   H, d          heads and head size; d in {32, 64, 128}; H >= 1.
+ *   total_tokens  rows of q, k, v and out.
+ *   max_seq_len   an upper bound on every L_b (sizes the schedule; a user longer than this
+ *                 is reported as HSTU_ERR_BAD_OFFSETS and skipped).
+ *   alpha         score scale inside the SiLU (finite).
+ *   N             output normaliser, one scalar for the whole call (finite, > 0).
+ *   out           device, bf16 [total_tokens, H, d]; must not overlap q, k or v.
+ *   stream        cudaStream_t as void*.
+ */
+hstu_status_t hstu_attn_fwd(const void* q, const void* k, const void* v,
+                            const int32_t* seq_offsets, const int32_t* num_targets,
+                            int32_t B, int32_t H, int32_t d,
+                            int32_t total_tokens, int32_t max_seq_len,
+                            float alpha, float N,
+                            void* out, void* stream);
+
+/*
+ * hstu_attn_fwd_cached — streaming variant: only the new tokens of each user are queried;
+ * keys and values cover the cached history prefix plus the new tokens (the K/V reuse across
+ * consecutive timestamps of the DLRMv3 review, section "model selection").
+ *
+ *   q             device, bf16 [total_q, H, d]: for each user, its new rows only, users
+ *                 packed in order (user b's new rows start at
+ *                 seq_offsets[b] - sum_{b' < b} cached_len[b']).
+ *   k, v          device, bf16 [total_kv, H, d]: full segments (cached prefix + new rows),
+ *                 jagged by seq_offsets exactly as in hstu_attn_fwd.
+ *   num_targets   as in hstu_attn_fwd (targets are the last T_b rows of the full segment).
+ *   cached_len    device, int32 [B]: 0 <= cached_len[b] <= U_b (the prefix is history only).
+ *                 NULL means all zero, which makes the call identical to hstu_attn_fwd.
+ *   total_q       must equal total_kv - sum_b cached_len[b] (checked on the device).
+ *   out           device, bf16 [total_q, H, d]: row r of user b is the output of position
+ *                 cached_len[b] + r, identical to that row of a full recomputation.
+ *   Other arguments as in hstu_attn_fwd.
+ */
+hstu_status_t hstu_attn_fwd_cached(const void* q, const void* k, const void* v,
+                                   const int32_t* seq_offsets, const int32_t* num_targets,
+                                   const int32_t* cached_len,
+                                   int32_t B, int32_t H, int32_t d,
+                                   int32_t total_kv, int32_t total_q, int32_t max_seq_len,
+                                   float alpha, float N,
+                                   void* out, void* stream);
+
+/*
+ * Two-step form.  hstu_attn_fwd / hstu_attn_fwd_cached are hstu_attn_plan followed by
+ * hstu_attn_fwd_planned on a buffer the library takes from its own pool.  Callers that run the
+ * attention several times over the same jagged structure (several layers, heads groups or
+ * repeated requests) can build the plan once and replay it; the plan is also what a caller
+ * inspects to see the work list.
+ *
+ * hstu_attn_plan_bytes — bytes of a plan buffer for (B, H, total_q) (0 for invalid sizes).
+ *   Layout (all int32, little endian):
+ *     header[4]          {work counter, num_items, finished-CTA counter, 0}
+ *     q_start[B]         first query row of each user (-1: user skipped), padded to 16 bytes
+ *     items[cap][4]      {b, pair, h, cost}, cap = H * (total_q / 256 + B); the first
+ *                        num_items entries are valid, in non-increasing cost order.  `pair` is
+ *                        a block of 256 query rows of user b; `cost` is the number of 128x128
+ *                        score tiles the block computes (fully masked tiles are not counted).
+ *
+ * hstu_attn_plan — validates the offsets on the device and writes the plan.
+ *   seq_offsets, num_targets, cached_len, B, H, total_kv, total_q, max_seq_len: as in
+ *   hstu_attn_fwd_cached (cached_len NULL and total_q = total_kv for a full pass).
+ *   plan         device, 16-byte aligned, plan_bytes >= hstu_attn_plan_bytes(B, H, total_q).
+ *
+ * hstu_attn_fwd_planned — the attention kernel over a plan built by hstu_attn_plan from the
+ *   same seq_offsets / num_targets / cached_len / B / H / total_q.  Arguments as in
+ *   hstu_attn_fwd_cached.  The kernel re-arms the plan's work counter when it finishes, so a
+ *   plan may be replayed any number of times on one stream; two calls that share a plan must
+ *   not overlap in time.
+ */
+int64_t hstu_attn_plan_bytes(int32_t B, int32_t H, int32_t total_q);
+
+hstu_status_t hstu_attn_plan(const int32_t* seq_offsets, const int32_t* num_targets,
+                             const int32_t* cached_len,
+                             int32_t B, int32_t H, int32_t total_kv, int32_t total_q,
+                             int32_t max_seq_len,
+                             void* plan, int64_t plan_bytes, void* stream);
+
+hstu_status_t hstu_attn_fwd_planned(const void* q, const void* k, const void* v,
+                                    const int32_t* seq_offsets, const int32_t* num_targets,
+                                    const int32_t* cached_len,
+                                    int32_t B, int32_t H, int32_t d,
+                                    int32_t total_kv, int32_t total_q,
+                                    float alpha, float N,
+                                    void* plan, void* out, void* stream);
+
+/*
+ * hstu_attn_get_error — synchronises `stream`, returns the device error word of the current
+ * device as a status (HSTU_OK if clean) and clears it.  The word is shared by all calls on
+ * the device, so a nonzero status may come from any call completed since the last read.
+ */
+hstu_status_t hstu_attn_get_error(void* stream);
+
+/* Static, human-readable name of a status. */
+const char* hstu_attn_status_string(hstu_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_ATTN_H_ */

@@ -1,0 +1,87 @@
+"""CPU: libhstu_attn.so builds for sm_100a, loads, and exports every function include/hstu_attn.h
+declares; host-side argument validation answers synchronously without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hstu_attn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hstu_attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    assert declared_functions() == sorted(["hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_plan_bytes",
+                                           "hstu_attn_plan", "hstu_attn_fwd_planned", "hstu_attn_get_error",
+                                           "hstu_attn_status_string"])
+
+
+def test_library_exports_every_declared_symbol(cuda_lib):
+    from hstu_pointwise_attention_jagged_b200 import binding
+    for name in declared_functions():
+        assert hasattr(cuda_lib, name), name
+    assert sorted(binding.EXPORTS) == declared_functions()
+    # the exported names are plain C symbols
+    out = os.popen("nm -D --defined-only %s" % binding.library_path()).read()
+    for name in declared_functions():
+        assert re.search(r"\sT %s$" % name, out, re.M), name
+
+
+def test_status_strings(cuda_lib):
+    names = [cuda_lib.hstu_attn_status_string(i).decode() for i in range(6)]
+    assert names == ["HSTU_OK", "HSTU_ERR_INVALID_ARGUMENT", "HSTU_ERR_UNSUPPORTED", "HSTU_ERR_CUDA",
+                     "HSTU_ERR_BAD_OFFSETS", "HSTU_ERR_TIMEOUT"]
+
+
+def test_plan_bytes(cuda_lib):
+    """16-byte header, B query-row starts padded to 16 bytes, 16 bytes per possible item."""
+    assert cuda_lib.hstu_attn_plan_bytes(8, 4, 32768) == 16 + 32 + 16 * 4 * (32768 // 256 + 8)
+    assert cuda_lib.hstu_attn_plan_bytes(3, 1, 10) == 16 + 16 + 16 * 3
+    assert cuda_lib.hstu_attn_plan_bytes(-1, 4, 10) == 0
+
+
+def _fwd(lib, **kw):
+    args = dict(q=1 << 12, k=1 << 12, v=1 << 12, off=1 << 12, nt=None, B=1, H=2, d=128, total=16,
+                msl=16, alpha=1.0, N=16.0, out=1 << 20, stream=None)
+    args.update(kw)
+    vp = ctypes.c_void_p
+    return lib.hstu_attn_fwd(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["off"]), vp(args["nt"]),
+                             args["B"], args["H"], args["d"], args["total"], args["msl"], args["alpha"], args["N"],
+                             vp(args["out"]), vp(args["stream"]))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(off=None), 1), (dict(out=None), 1), (dict(B=-1), 1), (dict(H=0), 1),
+    (dict(N=0.0), 1), (dict(N=float("nan")), 1), (dict(alpha=float("inf")), 1), (dict(total=-5), 1),
+    (dict(d=48), 2), (dict(d=256), 2), (dict(q=(1 << 12) + 8), 2), (dict(out=1 << 12), 1),
+])
+def test_host_validation(cuda_lib, kw, status):
+    """Rejected before any CUDA call: no GPU is needed to see these statuses."""
+    assert _fwd(cuda_lib, **kw) == status
+
+
+def test_host_validation_cached_and_planned(cuda_lib):
+    vp = ctypes.c_void_p
+    # total_q > total_kv is impossible
+    st = cuda_lib.hstu_attn_fwd_cached(vp(4096), vp(4096), vp(4096), vp(4096), None, None, 1, 1, 64, 10, 11, 10,
+                                       1.0, 1.0, vp(1 << 20), None)
+    assert st == 1
+    # a plan buffer smaller than hstu_attn_plan_bytes
+    st = cuda_lib.hstu_attn_plan(vp(4096), None, None, 2, 1, 10, 10, 10, vp(1 << 20), 16, None)
+    assert st == 1
+    # fwd_planned without a plan
+    st = cuda_lib.hstu_attn_fwd_planned(vp(4096), vp(4096), vp(4096), vp(4096), None, None, 1, 1, 64, 10, 10,
+                                        1.0, 1.0, None, vp(1 << 20), None)
+    assert st == 1
+
+
+def test_zero_rows_need_no_pointers(cuda_lib):
+    """With no query rows nothing is read or written: NULL token pointers are accepted."""
+    assert _fwd(cuda_lib, q=None, k=None, v=None, out=None, total=0, B=3) == 0
+    assert _fwd(cuda_lib, q=None, k=None, v=None, out=None, off=None, total=0, B=0) == 0

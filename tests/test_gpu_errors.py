@@ -1,0 +1,75 @@
+"""GPU: error reporting.  Inconsistent lengths are detected on the device, reported through
+hstu_attn_get_error, and the offending users are skipped while the others are computed; bad
+arguments are rejected synchronously."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import assert_parity, dev_bf16, dev_i32, to_f64
+from hstu_pointwise_attention_jagged_b200 import binding, workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def test_clean_call_reports_ok():
+    w = workloads.make_custom("ok", [100, 50], [3, 2], 2, 64, 0.125, 103.0, seed=31)
+    binding.hstu_attn_fwd(dev_bf16(w.q), dev_bf16(w.k), dev_bf16(w.v), dev_i32(w.seq_offsets),
+                          dev_i32(w.num_targets), w.alpha, w.N, w.max_seq_len)
+    assert binding.hstu_attn_get_error() == 0
+
+
+def test_bad_targets_skip_user_and_report():
+    """User 1 claims more candidates than tokens: it is skipped, users 0 and 2 are still right."""
+    w = workloads.make_custom("bad", [150, 60, 90], [10, 5, 4], 2, 128, 1 / math.sqrt(128), 160.0, seed=32)
+    bad_nt = w.num_targets.copy()
+    bad_nt[1] = 1000
+    out = torch.full((w.total, w.H, w.d), 5.0, dtype=torch.bfloat16, device="cuda")
+    binding.hstu_attn_fwd(dev_bf16(w.q), dev_bf16(w.k), dev_bf16(w.v), dev_i32(w.seq_offsets), dev_i32(bad_nt),
+                          w.alpha, w.N, w.max_seq_len, out=out)
+    assert binding.hstu_attn_get_error() == 4  # HSTU_ERR_BAD_OFFSETS
+    assert binding.hstu_attn_get_error() == 0  # cleared by the read
+    ref = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N)
+    o = to_f64(out)
+    s = w.seq_offsets
+    assert np.all(o[s[1]:s[2]] == 5.0)
+    keep = np.r_[s[0]:s[1], s[2]:s[3]]
+    assert_parity(o[keep], ref[keep], what="valid users")
+
+
+def test_user_longer_than_max_seq_len_is_skipped():
+    w = workloads.make_custom("long", [300, 20], [0, 0], 1, 64, 0.125, 300.0, seed=33)
+    out = torch.full((w.total, 1, 64), 5.0, dtype=torch.bfloat16, device="cuda")
+    binding.hstu_attn_fwd(dev_bf16(w.q), dev_bf16(w.k), dev_bf16(w.v), dev_i32(w.seq_offsets), None,
+                          w.alpha, w.N, 100, out=out)
+    assert binding.hstu_attn_get_error() == 4
+    assert torch.all(out[:300] == 5.0)
+    ref = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, None, w.alpha, w.N)
+    assert_parity(to_f64(out[300:]), ref[300:], what="short user")
+
+
+def test_cached_prefix_into_candidates_is_rejected():
+    w = workloads.make_custom("cbad", [100, 80], [20, 10], 1, 64, 0.125, 120.0, seed=34, cached_len=[0, 0])
+    cl = np.array([110, 0], np.int32)  # reaches into user 0's candidates
+    q_new = dev_bf16(w.q[np.r_[110:120, 120:210]])
+    out = torch.full((100, 1, 64), 5.0, dtype=torch.bfloat16, device="cuda")
+    binding.hstu_attn_fwd_cached(q_new, dev_bf16(w.k), dev_bf16(w.v), dev_i32(w.seq_offsets),
+                                 dev_i32(w.num_targets), dev_i32(cl), w.alpha, w.N, 120, out=out)
+    assert binding.hstu_attn_get_error() == 4
+
+
+def test_synchronous_argument_errors():
+    q = torch.zeros((16, 2, 48), dtype=torch.bfloat16, device="cuda")
+    off = torch.tensor([0, 16], dtype=torch.int32, device="cuda")
+    with pytest.raises(binding.HstuError) as e:
+        binding.hstu_attn_fwd(q, q, q, off, None, 1.0, 1.0, 16)
+    assert e.value.status == 2
+    q = torch.zeros((16, 2, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(binding.HstuError) as e:
+        binding.hstu_attn_fwd(q, q, q, off, None, 1.0, 0.0, 16)
+    assert e.value.status == 1
+    with pytest.raises(binding.HstuError) as e:
+        binding.hstu_attn_fwd(q, q, q, off, None, 1.0, 1.0, 16, out=q)
+    assert e.value.status == 1
