@@ -30,6 +30,7 @@ EXPORTS = (
     "hstu_attn_plan_bytes",
     "hstu_attn_plan",
     "hstu_attn_fwd_planned",
+    "hstu_attn_fwd_noalloc",
     "hstu_attn_get_error",
     "hstu_attn_status_string",
 )
@@ -65,6 +66,9 @@ def load_library():
     lib.hstu_attn_plan_bytes.restype = i64
     lib.hstu_attn_plan.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, i64, vp]
     lib.hstu_attn_fwd_planned.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp]
+    lib.hstu_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, f32,
+                                          vp, vp]
+    lib.hstu_attn_fwd_noalloc.restype = ctypes.c_int
     lib.hstu_attn_get_error.argtypes = [vp]
     lib.hstu_attn_status_string.argtypes = [ctypes.c_int]
     lib.hstu_attn_status_string.restype = ctypes.c_char_p
@@ -203,6 +207,32 @@ def hstu_attn_fwd_planned(q, k, v, seq_offsets, num_targets, cached_len, alpha, 
                                        _ptr(cached_len), B, H, d, total_kv, total_q, float(alpha), float(N),
                                        _ptr(plan), _ptr(out), _stream_ptr(stream, q.device))
     _raise_if(st, "hstu_attn_fwd_planned")
+    return out
+
+
+def hstu_attn_fwd_noalloc(q, k, v, seq_offsets, num_targets, cached_len, alpha, N, max_seq_len, out=None,
+                          stream=None):
+    """hstu_attn_fwd_cached whose plan lives in the library's fixed device array, for callers that
+    must not allocate device memory during a call (see include/hstu_attn.h for the size limit and
+    the rule that calls must not overlap on the GPU).  Pass cached_len=None for a full pass."""
+    lib = load_library()
+    _check_tokens("q", q)
+    total_q, H, d = q.shape
+    _check_tokens("k", k, H, d)
+    _check_tokens("v", v, H, d)
+    total_kv = k.shape[0]
+    B = seq_offsets.numel() - 1
+    _check_index("seq_offsets", seq_offsets, B + 1, q.device, optional=False)
+    _check_index("num_targets", num_targets, B, q.device)
+    _check_index("cached_len", cached_len, B, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tokens("out", out, H, d)
+    with torch.cuda.device(q.device):
+        st = lib.hstu_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(num_targets),
+                                       _ptr(cached_len), B, H, d, total_kv, total_q, int(max_seq_len),
+                                       float(alpha), float(N), _ptr(out), _stream_ptr(stream, q.device))
+    _raise_if(st, "hstu_attn_fwd_noalloc")
     return out
 
 

@@ -265,6 +265,45 @@ hstu_status_t run(const void* q, const void* k, const void* v, const int32_t* se
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------------------------------------
+// Allocation-free variant (hstu_attn_fwd_noalloc).  Its plan lives in this fixed device array
+// instead of a buffer from the memory pool.  Every device that loads the library holds the
+// array until the process exits.  In host code `g_noalloc_plan` names a host-side stand-in, not
+// device memory, so the kernels get the device address that cudaGetSymbolAddress returns.
+static __device__ __align__(256) unsigned char g_noalloc_plan[HSTU_ATTN_NOALLOC_PLAN_BYTES];
+
+namespace {
+
+struct NoAllocState {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  DeviceState dev;        // SM count and error word only; its memory pool is never created
+  void* plan = nullptr;   // device address of g_noalloc_plan on this device
+};
+NoAllocState g_noalloc[kMaxDevices];
+
+// Runs once per device, with that device current: looks up the device addresses of the plan
+// array and of the error word and sets the kernels' shared-memory limits.  Allocates nothing.
+void init_noalloc(NoAllocState& na, int dev) {
+  cudaError_t e = cudaDeviceGetAttribute(&na.dev.num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaGetSymbolAddress(&na.plan, g_noalloc_plan);
+  if (e == cudaSuccess) e = cudaGetSymbolAddress(reinterpret_cast<void**>(&na.dev.err_word), g_error_word);
+  if (e == cudaSuccess) e = set_kernel_attrs<32>();
+  if (e == cudaSuccess) e = set_kernel_attrs<64>();
+  if (e == cudaSuccess) e = set_kernel_attrs<128>();
+  na.err = e;
+}
+
+NoAllocState* noalloc_state() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  NoAllocState& na = g_noalloc[dev];
+  std::call_once(na.once, init_noalloc, std::ref(na), dev);
+  return na.err == cudaSuccess ? &na : nullptr;
+}
+
+}  // namespace
 }  // namespace hstu
 
 extern "C" {
@@ -347,6 +386,29 @@ const char* hstu_attn_status_string(hstu_status_t s) {
     case HSTU_ERR_TIMEOUT: return "HSTU_ERR_TIMEOUT";
   }
   return "HSTU_ERR_UNKNOWN";
+}
+
+hstu_status_t hstu_attn_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* seq_offsets,
+                                    const int32_t* num_targets, const int32_t* cached_len, int32_t B, int32_t H,
+                                    int32_t d, int32_t total_kv, int32_t total_q, int32_t max_seq_len, float alpha,
+                                    float N, void* out, void* stream_ptr) {
+  hstu_status_t s = hstu::check_sizes(B, H, total_kv, total_q);
+  if (s == HSTU_OK && max_seq_len < 0) s = HSTU_ERR_INVALID_ARGUMENT;
+  if (s == HSTU_OK) s = hstu::check_tokens(q, k, v, seq_offsets, H, d, total_kv, total_q, alpha, N, out);
+  if (s != HSTU_OK) return s;
+  if (hstu::plan_bytes(B, H, total_q) > static_cast<int64_t>(HSTU_ATTN_NOALLOC_PLAN_BYTES))
+    return HSTU_ERR_UNSUPPORTED;  // the batch needs a bigger plan than the fixed array holds
+  if (B == 0 || total_q == 0) return HSTU_OK;
+  hstu::NoAllocState* na = hstu::noalloc_state();
+  if (!na) return HSTU_ERR_CUDA;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  // The plan kernel rewrites every plan word the attention kernel reads (header counters
+  // included), so what an earlier call left in the array does not matter.
+  if (hstu::launch_plan(seq_offsets, num_targets, cached_len, B, H, total_kv, total_q, max_seq_len,
+                        hstu::carve(na->plan, B), na->dev.err_word, stream) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  return hstu::launch_attention(&na->dev, q, k, v, seq_offsets, num_targets, cached_len, B, H, d, total_kv,
+                                total_q, alpha, N, na->plan, out, stream);
 }
 
 }  // extern "C"

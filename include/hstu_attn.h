@@ -167,6 +167,42 @@ hstu_status_t hstu_attn_fwd_planned(const void* q, const void* k, const void* v,
                                     void* plan, void* out, void* stream);
 
 /*
+ * hstu_attn_fwd_noalloc — hstu_attn_fwd_cached without any device-memory allocation.  (An
+ * addition of this library for its callers; the pages describe no such call.)
+ *
+ * Why: some callers cannot allocate device memory while they run a batch — serving processes
+ * that reserve all of the GPU's memory up front for their own caching allocator, or code on a
+ * latency-critical path where an allocator call may block or synchronise.  Every other entry
+ * point either takes its plan buffer from the library's memory pool or wants the caller to
+ * provide one; this one keeps the plan in a fixed array of HSTU_ATTN_NOALLOC_PLAN_BYTES bytes
+ * that is part of the library's device image.
+ *
+ *   Arguments are those of hstu_attn_fwd_cached (cached_len = NULL and total_q = total_kv for a
+ *   full pass).  The caller still provides q, k, v and out.
+ *   Limit: hstu_attn_plan_bytes(B, H, total_q) must not exceed HSTU_ATTN_NOALLOC_PLAN_BYTES
+ *   (1 MiB: about 65,000 work items of 256 query rows x 1 head, e.g. H = 8 and 2 million query
+ *   rows); larger batches return HSTU_ERR_UNSUPPORTED before anything is launched.
+ *   Memory: every GPU that loads the library holds the 1 MiB array until the process exits.
+ *   First call: the first call on each device (with that device current) looks up the array's
+ *   device address once; make that first call before any stream capture.
+ *   Sharing: all calls on a device use the same array.  Calls whose GPU work overlaps in time
+ *   (different streams, or different host threads without ordering) race on it and may produce
+ *   wrong outputs; order them on one stream or with events.  Each call rewrites the part of the
+ *   array it reads, so leftovers from earlier calls are harmless.
+ *   Returns, besides the statuses of hstu_attn_fwd_cached, HSTU_ERR_UNSUPPORTED for a batch over
+ *   the limit.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define HSTU_ATTN_NOALLOC_PLAN_BYTES (1u << 20)
+
+hstu_status_t hstu_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                    const int32_t* seq_offsets, const int32_t* num_targets,
+                                    const int32_t* cached_len,
+                                    int32_t B, int32_t H, int32_t d,
+                                    int32_t total_kv, int32_t total_q, int32_t max_seq_len,
+                                    float alpha, float N,
+                                    void* out, void* stream);
+
+/*
  * hstu_attn_get_error — synchronises `stream`, returns the device error word of the current
  * device as a status (HSTU_OK if clean) and clears it.  The word is shared by all calls on
  * the device, so a nonzero status may come from any call completed since the last read.

@@ -18,8 +18,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     assert declared_functions() == sorted(["hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_plan_bytes",
-                                           "hstu_attn_plan", "hstu_attn_fwd_planned", "hstu_attn_get_error",
-                                           "hstu_attn_status_string"])
+                                           "hstu_attn_plan", "hstu_attn_fwd_planned", "hstu_attn_fwd_noalloc",
+                                           "hstu_attn_get_error", "hstu_attn_status_string"])
 
 
 def test_library_exports_every_declared_symbol(cuda_lib):
