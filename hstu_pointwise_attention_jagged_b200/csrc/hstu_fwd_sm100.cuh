@@ -53,9 +53,9 @@ struct FwdCfg {
   static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, true);
 };
 
-constexpr int kNumThreads = 320;  // 8 SiLU warps + producer + MMA
+constexpr int kNumThreads = 320;  // 8 SiLU warps + producer + MMA issuer
 constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;       // issues every MMA and owns the TMEM allocation
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s per wait
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s per drain wait on the abort path
 
@@ -105,10 +105,9 @@ __device__ __forceinline__ Work read_slot(const volatile int32_t* s) {
   return w;
 }
 
-// Waits for phase `parity` of `bar`; false if the CTA is aborting or this wait timed out.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag,
-                                          unsigned* err) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
+// Slow path of wait_bounded: spins until the phase completes, the CTA aborts, or the time limit.
+__device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag,
+                                               unsigned* err) {
   const uint64_t t0 = ptx::globaltimer_ns();
   while (true) {
 #pragma unroll 1
@@ -121,6 +120,14 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
       return false;
     }
   }
+}
+
+// Waits for phase `parity` of `bar`; false if the CTA is aborting or this wait timed out.  The
+// first test is inline: a call right after a burst of MMAs stalls the issuing warp.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag,
+                                             unsigned* err) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  return wait_bounded_slow(bar, parity, abort_flag, err);
 }
 
 // Abort-path drain: waits for phase `parity` of `bar` for at most kDrainLimitNs.
@@ -187,9 +194,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
     for (int h = 0; h < 2; ++h) {
       ptx::mbar_init(bar(ctl->s_full[h]), 1);
-      ptx::mbar_init(bar(ctl->p_full[h]), 128);
+      ptx::mbar_init(bar(ctl->p_full[h]), 4);   // one arrival per SiLU warp
       ptx::mbar_init(bar(ctl->o_full[h]), 1);
-      ptx::mbar_init(bar(ctl->o_empty[h]), 128);
+      ptx::mbar_init(bar(ctl->o_empty[h]), 4);
       ptx::mbar_init(bar(ctl->sched_full[h]), 1);
       ptx::mbar_init(bar(ctl->sched_empty[h]), 1 + 8);
     }
@@ -291,6 +298,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      // Descriptor templates: the descriptor of address a + off is template(a) + (off >> 4).
+      const uint64_t dq0 = ptx::smem_desc(sQ, 16, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
+      const uint64_t dk0 = ptx::smem_desc(sKV, 16, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
+      const uint64_t dv0 = ptx::smem_desc(sKV, Cfg::kBlockBytes, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
       int slot = 0;
       uint32_t sched_full_par[2] = {0u, 0u};
       uint32_t q_full_par = 0u;
@@ -298,32 +309,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       uint32_t o_empty_par[2] = {1u, 1u};
       int stage = 0;
       uint32_t kv_phase = 0;
-      const uint32_t colS[2] = {Cfg::kColS0, Cfg::kColS1};
-      const uint32_t colO[2] = {Cfg::kColO0, Cfg::kColO1};
       bool ok = true;
-
-      auto issue_s = [&](int hh, int st) {
-        const uint32_t qa = sQ + hh * Cfg::kTileBytes;
-        const uint32_t ka = sKV + st * Cfg::kTileBytes;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks / Cfg::kKStepsPerBlock) * Cfg::kBlockBytes + (ks % Cfg::kKStepsPerBlock) * 32;
-          const uint64_t da = ptx::smem_desc(qa + off, 16, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
-          const uint64_t db = ptx::smem_desc(ka + off, 16, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
-          ptx::mma_ss(tmem + colS[hh], da, db, Cfg::kIdescQK, ks > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int hh, int st, bool first) {
-        const uint32_t va = sKV + st * Cfg::kTileBytes;
-#pragma unroll
-        for (int ks = 0; ks < kTileRows / 16; ++ks) {
-          const uint64_t db = ptx::smem_desc(va + ks * 16 * Cfg::kRowBytes, Cfg::kBlockBytes,
-                                             8 * Cfg::kRowBytes, Cfg::kSwizzle);
-          ptx::mma_ts(tmem + colO[hh], tmem + colS[hh] + ks * 8, db, Cfg::kIdescPV,
-                      (first && ks == 0) ? 0u : 1u);
-        }
-      };
-
       while (ok) {
         if (!wait_bounded(bar(ctl->sched_full[slot]), sched_full_par[slot], abort_flag, p.err)) break;
         sched_full_par[slot] ^= 1u;
@@ -335,6 +321,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const TileRange un = key_tiles(w.pos0, w.pos0 + w.nrows, w.U);
         TileRange hr[2];
         int remaining[2];
+#pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int lo = hh * kTileRows;
           const int hi = w.nrows < lo + kTileRows ? w.nrows : lo + kTileRows;
@@ -350,63 +337,71 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         bool first[2] = {true, true};
         int prev_vst = 0;
         uint32_t prev_vph = 0;
-        bool v_waited = false;
-
-        // Issues the P.V MMA of half hh for the previous key tile (whose V sits in prev_vst).
-        auto flush_pv = [&](int hh) -> bool {
-          if (!wait_bounded(bar(ctl->p_full[hh]), p_full_par[hh], abort_flag, p.err)) return false;
-          p_full_par[hh] ^= 1u;
-          if (!v_waited) {
-            if (!wait_bounded(bar(ctl->kv_full[prev_vst]), prev_vph, abort_flag, p.err)) return false;
-            v_waited = true;
+        // Step i, per half in turn: the P.V of the previous key tile (if that half used it), then
+        // the scores of key tile i (if that half needs it).  The tensor pipe therefore alternates
+        // [P.V_0, S_0], [P.V_1, S_1], and one half's SiLU overlaps the other half's MMAs.  The
+        // extra last step only drains the P.V.
+        for (int i = 0; i <= n_u; ++i) {
+          const bool last = (i == n_u);
+          int t = 0, kst = 0, vst = 0;
+          uint32_t kph = 0, vph = 0;
+          if (!last) {
+            t = tile_at(un, i);
+            kst = stage;
+            kph = kv_phase;
+            if (++stage == Cfg::kStages) { stage = 0; kv_phase ^= 1u; }
+            vst = stage;
+            vph = kv_phase;
+            if (++stage == Cfg::kStages) { stage = 0; kv_phase ^= 1u; }
           }
-          if (first[hh]) {
-            if (!wait_bounded(bar(ctl->o_empty[hh]), o_empty_par[hh], abort_flag, p.err)) return false;
-            o_empty_par[hh] ^= 1u;
-          }
-          ptx::tc_fence_after();
-          issue_pv(hh, prev_vst, first[hh]);
-          first[hh] = false;
-          pend[hh] = false;
-          if (--remaining[hh] == 0) ptx::mma_commit(bar(ctl->o_full[hh]));
-          return true;
-        };
-
-        for (int i = 0; i < n_u && ok; ++i) {
-          const int t = tile_at(un, i);
-          const int kst = stage;
-          const uint32_t kph = kv_phase;
-          if (++stage == Cfg::kStages) { stage = 0; kv_phase ^= 1u; }
-          const int vst = stage;
-          const uint32_t vph = kv_phase;
-          if (++stage == Cfg::kStages) { stage = 0; kv_phase ^= 1u; }
-          bool k_waited = false;
-          for (int hh = 0; hh < 2 && ok; ++hh) {
-            if (pend[hh] && !flush_pv(hh)) { ok = false; break; }
-            if (tile_in(hr[hh], t)) {
+          bool k_waited = false, v_waited = false;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t colS = hh ? Cfg::kColS1 : Cfg::kColS0;
+            if (pend[hh]) {
+              ok = wait_bounded(bar(ctl->p_full[hh]), p_full_par[hh], abort_flag, p.err) &&
+                   (v_waited || wait_bounded(bar(ctl->kv_full[prev_vst]), prev_vph, abort_flag, p.err)) &&
+                   (!first[hh] || wait_bounded(bar(ctl->o_empty[hh]), o_empty_par[hh], abort_flag, p.err));
+              if (!ok) break;
+              v_waited = true;
+              p_full_par[hh] ^= 1u;
+              if (first[hh]) o_empty_par[hh] ^= 1u;
+              ptx::tc_fence_after();
+              const uint64_t dv = dv0 + ((prev_vst * Cfg::kTileBytes) >> 4);
+              const uint32_t colO = hh ? Cfg::kColO1 : Cfg::kColO0;
+#pragma unroll
+              for (int ks = 0; ks < kTileRows / 16; ++ks)
+                ptx::mma_ts(tmem + colO, tmem + colS + ks * 8, dv + ((ks * 16 * Cfg::kRowBytes) >> 4),
+                            Cfg::kIdescPV, (first[hh] && ks == 0) ? 0u : 1u);
+              first[hh] = false;
+              pend[hh] = false;
+              if (--remaining[hh] == 0) ptx::mma_commit(bar(ctl->o_full[hh]));
+            }
+            if (!last && tile_in(hr[hh], t)) {
               if (!k_waited) {
                 if (!wait_bounded(bar(ctl->kv_full[kst]), kph, abort_flag, p.err)) { ok = false; break; }
                 ptx::tc_fence_after();
                 k_waited = true;
               }
-              issue_s(hh, kst);
+              const uint64_t dq = dq0 + ((hh * Cfg::kTileBytes) >> 4);
+              const uint64_t dk = dk0 + ((kst * Cfg::kTileBytes) >> 4);
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t off =
+                    (ks / Cfg::kKStepsPerBlock) * Cfg::kBlockBytes + (ks % Cfg::kKStepsPerBlock) * 32;
+                ptx::mma_ss(tmem + colS, dq + (off >> 4), dk + (off >> 4), Cfg::kIdescQK, ks > 0 ? 1u : 0u);
+              }
               ptx::mma_commit(bar(ctl->s_full[hh]));
               pend[hh] = true;
             }
           }
           if (!ok) break;
-          ptx::mma_commit(bar(ctl->kv_empty[kst]));
-          if (i > 0) ptx::mma_commit(bar(ctl->kv_empty[prev_vst]));
-          if (i == n_u - 1) ptx::mma_commit(bar(ctl->q_empty));
+          if (!last) ptx::mma_commit(bar(ctl->kv_empty[kst]));       // K_t: free after its S MMAs
+          if (i > 0) ptx::mma_commit(bar(ctl->kv_empty[prev_vst]));  // V_{t-1}: free after its P.V
+          if (i == n_u - 1) ptx::mma_commit(bar(ctl->q_empty));      // Q: free after the last S MMA
           prev_vst = vst;
           prev_vph = vph;
-          v_waited = false;
         }
-        if (!ok) break;
-        for (int hh = 0; hh < 2; ++hh)
-          if (pend[hh] && !flush_pv(hh)) { ok = false; break; }
-        if (!ok) break;
-        if (n_u > 0) ptx::mma_commit(bar(ctl->kv_empty[prev_vst]));
       }
       // Every MMA this thread issued has completed once `drain` flips.
       ptx::mma_commit(bar(ctl->drain));
@@ -456,6 +451,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const bool full = (j0 + kTileRows <= w.U) && (j0 + kTileRows <= p0 + 1);
         const int lim = lim_abs - j0;
         const int self = i_pos - j0;
+        // 32-column chunks: the load of chunk c+1 is in flight while chunk c is computed.
         uint32_t ra[32], rb[32];
         ptx::tmem_ld32(taddr_s + 0, ra);
         ptx::tmem_ld_wait(ra);
@@ -471,7 +467,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         silu_chunk<3>(rb, taddr_s, half_alpha, full, lim, self);
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(ctl->p_full[hh]));
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(ctl->p_full[hh]));
       }
       if (!ok) break;
       // Epilogue: O_h * (1/N) -> bf16 -> out rows that exist.
@@ -500,7 +497,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         }
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(bar(ctl->o_empty[hh]));
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(ctl->o_empty[hh]));
     }
   }
 
