@@ -241,8 +241,9 @@ def plan_contents(plan, B):
     raw = plan.cpu().numpy().view("<i4")
     header = raw[:4].copy()
     qs_words = ((B * 4 + 15) // 16) * 4
+    ps_words = (((B + 1) * 4 + 15) // 16) * 4
     q_start = raw[4:4 + B].copy()
-    items = raw[4 + qs_words:].reshape(-1, 4)[:int(header[1])].copy()
+    items = raw[4 + qs_words + ps_words:].reshape(-1, 4)[:int(header[1])].copy()
     return header, q_start, items
 
 

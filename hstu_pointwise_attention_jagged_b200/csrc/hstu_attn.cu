@@ -112,21 +112,25 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 // Plan layout (documented in include/hstu_attn.h):
 //   int32 header[4] = {work counter, num_items, done counter, 0}
 //   int32 q_start[B], padded to 16 bytes
+//   int32 pair_start[B+1], padded to 16 bytes
 //   int4  items[capacity] = {b, pair, h, cost}, capacity = H * (total_q / 256 + B)
 struct Plan {
   int32_t* counter;
   int32_t* num_items;
   int32_t* done;
   int32_t* q_start;
+  int32_t* pair_start;
   int4* items;
 };
+
+size_t pad16(size_t n_ints) { return ((n_ints * 4 + 15) / 16) * 16; }
 
 int64_t capacity(int32_t B, int32_t H, int32_t total_q) {
   return static_cast<int64_t>(H) * (total_q / kPairRows + B);
 }
 
 int64_t plan_bytes(int32_t B, int32_t H, int32_t total_q) {
-  return 16 + ((static_cast<int64_t>(B) * 4 + 15) / 16) * 16 + capacity(B, H, total_q) * 16;
+  return 16 + static_cast<int64_t>(pad16(B) + pad16(static_cast<size_t>(B) + 1)) + capacity(B, H, total_q) * 16;
 }
 
 Plan carve(void* base, int32_t B) {
@@ -136,7 +140,8 @@ Plan carve(void* base, int32_t B) {
   w.num_items = reinterpret_cast<int32_t*>(p + 4);
   w.done = reinterpret_cast<int32_t*>(p + 8);
   w.q_start = reinterpret_cast<int32_t*>(p + 16);
-  w.items = reinterpret_cast<int4*>(p + 16 + ((static_cast<size_t>(B) * 4 + 15) / 16) * 16);
+  w.pair_start = reinterpret_cast<int32_t*>(p + 16 + pad16(B));
+  w.items = reinterpret_cast<int4*>(p + 16 + pad16(B) + pad16(static_cast<size_t>(B) + 1));
   return w;
 }
 
@@ -184,6 +189,7 @@ cudaError_t launch_plan(const int32_t* seq_offsets, const int32_t* num_targets, 
   a.nbins = cost_bins(max_seq_len);
   a.max_items = static_cast<int32_t>(capacity(B, H, total_q));
   a.q_start = w.q_start;
+  a.pair_start = w.pair_start;
   a.items = w.items;
   a.num_items = w.num_items;
   a.work_counter = w.counter;
@@ -193,11 +199,24 @@ cudaError_t launch_plan(const int32_t* seq_offsets, const int32_t* num_targets, 
   return cudaGetLastError();
 }
 
+// Launched as a programmatic dependent of the preceding kernel on the stream: its prologue
+// (barriers, TMEM allocation, tensor-map prefetch) overlaps the plan kernel, and the producer
+// waits for the preceding grid (griddepcontrol.wait) before its first global read.
 template <int D>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                        int grid, cudaStream_t stream) {
-  hstu_fwd_kernel<D><<<grid, kNumThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kNumThreads);
+  cfg.dynamicSmemBytes = FwdCfg<D>::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, hstu_fwd_kernel<D>, tq, tk, tv, p);
 }
 
 // The attention kernel over a plan built for the same offsets.  Arguments already checked.

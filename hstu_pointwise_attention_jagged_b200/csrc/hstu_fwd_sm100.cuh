@@ -219,6 +219,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
+      // Everything before this point touched only shared memory, TMEM and kernel parameters; the
+      // plan (and q/k/v) come from the preceding grid.
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       const int M = *p.num_items;
       int slot = 0;
       uint32_t sched_empty_par[2] = {1u, 1u};

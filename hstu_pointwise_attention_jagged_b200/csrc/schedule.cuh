@@ -80,6 +80,7 @@ struct SchedArgs {
   const int32_t* cached_len;   // [B] or null
   int32_t B, H, total_kv, total_q, max_seq_len, nbins, max_items;
   int32_t* q_start;       // [B] out: first query row of each user, -1 if the user is skipped
+  int32_t* pair_start;    // [B+1] out: index of each user's first 256-row block among all blocks
   int4* items;            // [max_items] out: {b, pair, h, cost}, non-increasing cost
   int32_t* num_items;     // [1] out
   int32_t* work_counter;  // [1] out: reset to 0 for the attention kernel's dynamic scheduler
@@ -115,68 +116,97 @@ __device__ __forceinline__ long long block_inclusive_scan(long long v, long long
   return v;
 }
 
+// User owning block g: the last b with pair_start[b] <= g (users without blocks share a start).
+__device__ __forceinline__ int owner_of(const int32_t* pair_start, int B, int g) {
+  int lo = 0, hi = B;  // pair_start[lo] <= g < pair_start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (pair_start[mid] <= g) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
 // One CTA of kSchedThreads threads.  Validates every user, assigns query-row starts, and writes
 // the work items sorted by non-increasing cost (counting sort over cost bins; ties in any order).
+// The per-block passes run one thread per (user, 256-row block).
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs a) {
+  // A dependent attention kernel may start its prologue now; it waits for this grid's writes
+  // (griddepcontrol.wait) before it reads anything in global memory.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ int hist[kMaxCostBins];
   __shared__ long long scan_scratch[32];
-  __shared__ long long carry_s;
+  __shared__ long long carry_q, carry_p;
   const int tid = threadIdx.x;
   const int nbins = a.nbins;
 
   for (int i = tid; i < nbins; i += kSchedThreads) hist[i] = 0;
   if (tid == 0) {
-    carry_s = 0;
+    carry_q = 0;
+    carry_p = 0;
     if (a.seq_offsets[0] != 0 || a.seq_offsets[a.B] != a.total_kv) atomicOr(a.err, kErrBadOffsets);
   }
   __syncthreads();
 
-  // Pass 1: per-user validation, query-row starts (exclusive prefix sum of new rows), cost
-  // histogram.
+  // Pass 1: per-user validation; one scan gives both the query-row starts (the caller's layout)
+  // and the block starts.
   for (int base = 0; base < a.B; base += kSchedThreads) {
     const int b = base + tid;
-    long long nq = 0;  // query rows this user occupies in the caller's q / out layout
+    long long nq = 0, npairs = 0;  // rows in the layout; 256-row blocks to compute
     bool ok = false;
-    int L = 0, T = 0, c = 0;
     if (b < a.B) {
       const int o0 = a.seq_offsets[b], o1 = a.seq_offsets[b + 1];
-      L = o1 - o0;
-      T = a.num_targets ? a.num_targets[b] : 0;
-      c = a.cached_len ? a.cached_len[b] : 0;
-      ok = o0 >= 0 && L >= 0 && o1 <= a.total_kv && L <= a.max_seq_len && T >= 0 && T <= L &&
-           c >= 0 && c <= L - T;
+      const int L = o1 - o0;
+      const int T = a.num_targets ? a.num_targets[b] : 0;
+      const int c = a.cached_len ? a.cached_len[b] : 0;
+      ok = o0 >= 0 && L >= 0 && o1 <= a.total_kv && L <= a.max_seq_len && T >= 0 && T <= L && c >= 0 &&
+           c <= L - T;
       if (!ok) atomicOr(a.err, kErrBadOffsets);
       // A skipped user still owns its rows of the layout, so later users keep their places.
       const int cc = c < 0 ? 0 : c;
       nq = L > cc ? (long long)(L - cc) : 0;
+      npairs = ok ? cdiv(L - c, kPairRows) : 0;
     }
     long long tot;
-    const long long incl = block_inclusive_scan(nq, scan_scratch, &tot);
-    const long long start = carry_s + incl - nq;
+    const long long incl = block_inclusive_scan((nq << 32) | npairs, scan_scratch, &tot);
+    const long long start_q = carry_q + (incl >> 32) - nq;
+    const long long start_p = carry_p + (incl & 0xffffffffll) - npairs;
     if (b < a.B) {
-      if (ok && start + nq > a.total_q) {
+      if (ok && start_q + nq > a.total_q) {
         ok = false;
         atomicOr(a.err, kErrBadOffsets);
       }
-      a.q_start[b] = ok ? (int)start : -1;
-      if (ok) {
-        const int U = L - T;
-        const int npairs = cdiv(L - c, kPairRows);
-        for (int p = 0; p < npairs; ++p) {
-          const int rows = (L - c) - p * kPairRows;
-          int cost = pair_cost(c + p * kPairRows, rows < kPairRows ? rows : kPairRows, U);
-          cost = cost < nbins ? cost : nbins - 1;
-          atomicAdd(&hist[cost], a.H);
-        }
-      }
+      a.q_start[b] = ok ? (int)start_q : -1;
+      a.pair_start[b] = (int)start_p;
     }
     __syncthreads();
-    if (tid == 0) carry_s += tot;
+    if (tid == 0) {
+      carry_q += tot >> 32;
+      carry_p += tot & 0xffffffffll;
+    }
     __syncthreads();
   }
-  if (tid == 0 && carry_s != a.total_q) atomicOr(a.err, kErrBadOffsets);
+  const int npairs_total = (int)carry_p;
+  if (tid == 0) {
+    a.pair_start[a.B] = npairs_total;
+    if (carry_q != a.total_q) atomicOr(a.err, kErrBadOffsets);
+  }
+  __syncthreads();
 
-  // Pass 2: bin start = number of items in strictly costlier bins (descending order).
+  // Pass 2: cost histogram, one thread per block.
+  for (int g = tid; g < npairs_total; g += kSchedThreads) {
+    const int b = owner_of(a.pair_start, a.B, g);
+    if (a.q_start[b] < 0) continue;
+    const int L = a.seq_offsets[b + 1] - a.seq_offsets[b];
+    const int U = L - (a.num_targets ? a.num_targets[b] : 0);
+    const int c = a.cached_len ? a.cached_len[b] : 0;
+    const int pr = g - a.pair_start[b];
+    const int rows = (L - c) - pr * kPairRows;
+    const int cost = pair_cost(c + pr * kPairRows, rows < kPairRows ? rows : kPairRows, U);
+    atomicAdd(&hist[cost < nbins ? cost : nbins - 1], a.H);
+  }
+  __syncthreads();
+
+  // Pass 3: bin start = number of items in strictly costlier bins (descending order).
   const int per = cdiv(nbins, kSchedThreads);
   long long part = 0;
   for (int k = 0; k < per; ++k) {
@@ -202,23 +232,19 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
     *a.done_counter = 0;
   }
 
-  // Pass 3: scatter items into their bins.
-  for (int b = tid; b < a.B; b += kSchedThreads) {
-    const int qs = a.q_start[b];
-    if (qs < 0) continue;
+  // Pass 4: scatter the items into their bins, one thread per block.
+  for (int g = tid; g < npairs_total; g += kSchedThreads) {
+    const int b = owner_of(a.pair_start, a.B, g);
+    if (a.q_start[b] < 0) continue;
     const int L = a.seq_offsets[b + 1] - a.seq_offsets[b];
-    const int T = a.num_targets ? a.num_targets[b] : 0;
+    const int U = L - (a.num_targets ? a.num_targets[b] : 0);
     const int c = a.cached_len ? a.cached_len[b] : 0;
-    const int U = L - T;
-    const int npairs = cdiv(L - c, kPairRows);
-    for (int p = 0; p < npairs; ++p) {
-      const int rows = (L - c) - p * kPairRows;
-      const int cost = pair_cost(c + p * kPairRows, rows < kPairRows ? rows : kPairRows, U);
-      const int bin = cost < nbins ? cost : nbins - 1;
-      const int pos = atomicAdd(&hist[bin], a.H);
-      for (int h = 0; h < a.H; ++h)
-        if (pos + h < a.max_items) a.items[pos + h] = make_int4(b, p, h, cost);
-    }
+    const int pr = g - a.pair_start[b];
+    const int rows = (L - c) - pr * kPairRows;
+    const int cost = pair_cost(c + pr * kPairRows, rows < kPairRows ? rows : kPairRows, U);
+    const int pos = atomicAdd(&hist[cost < nbins ? cost : nbins - 1], a.H);
+    for (int h = 0; h < a.H; ++h)
+      if (pos + h < a.max_items) a.items[pos + h] = make_int4(b, pr, h, cost);
   }
 }
 

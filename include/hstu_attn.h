@@ -134,6 +134,7 @@ hstu_status_t hstu_attn_fwd_cached(const void* q, const void* k, const void* v,
  *   Layout (all int32, little endian):
  *     header[4]          {work counter, num_items, finished-CTA counter, 0}
  *     q_start[B]         first query row of each user (-1: user skipped), padded to 16 bytes
+ *     pair_start[B+1]    index of each user's first 256-row block, padded to 16 bytes
  *     items[cap][4]      {b, pair, h, cost}, cap = H * (total_q / 256 + B); the first
  *                        num_items entries are valid, in non-increasing cost order.  `pair` is
  *                        a block of 256 query rows of user b; `cost` is the number of 128x128
