@@ -300,116 +300,124 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      // Descriptor templates: the descriptor of address a + off is template(a) + (off >> 4).
-      const uint64_t dq0 = ptx::smem_desc(sQ, 16, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
-      const uint64_t dk0 = ptx::smem_desc(sKV, 16, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
-      const uint64_t dv0 = ptx::smem_desc(sKV, Cfg::kBlockBytes, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
-      int slot = 0;
-      uint32_t sched_full_par[2] = {0u, 0u};
-      uint32_t q_full_par = 0u;
-      uint32_t p_full_par[2] = {0u, 0u};
-      uint32_t o_empty_par[2] = {1u, 1u};
-      int stage = 0;
-      uint32_t kv_phase = 0;
-      bool ok = true;
-      while (ok) {
-        if (!wait_bounded(bar(ctl->sched_full[slot]), sched_full_par[slot], abort_flag, p.err)) break;
-        sched_full_par[slot] ^= 1u;
-        const Work w = read_slot(ctl->slot[slot]);
-        ptx::mbar_arrive(bar(ctl->sched_empty[slot]));
-        slot ^= 1;
-        if (!w.valid) break;
+    // The whole warp runs this loop in step, so the control flow is uniform and the descriptors
+    // and TMEM addresses stay in uniform registers; lane 0 alone issues the tcgen05 instructions
+    // (the *_lead forms), so every MMA and commit comes from one thread, as commit tracking needs.
+    const uint32_t lead = (lane == 0) ? 1u : 0u;
+    // Waits are taken by every lane and the outcome is made warp-uniform.
+    auto wait_all = [&](uint32_t b, uint32_t par) {
+      return __all_sync(0xffffffffu, wait_bounded(b, par, abort_flag, p.err));
+    };
+    // Descriptor templates: the descriptor of address a + off is template(a) + (off >> 4).
+    const uint64_t dq0 = ptx::smem_desc(sQ, 16, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
+    const uint64_t dk0 = ptx::smem_desc(sKV, 16, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
+    const uint64_t dv0 = ptx::smem_desc(sKV, Cfg::kBlockBytes, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
+    int slot = 0;
+    uint32_t sched_full_par[2] = {0u, 0u};
+    uint32_t q_full_par = 0u;
+    uint32_t p_full_par[2] = {0u, 0u};
+    uint32_t o_empty_par[2] = {1u, 1u};
+    int stage = 0;
+    uint32_t kv_phase = 0;
+    bool ok = true;
+    while (ok) {
+      if (!wait_all(bar(ctl->sched_full[slot]), sched_full_par[slot])) break;
+      sched_full_par[slot] ^= 1u;
+      const Work w = read_slot(ctl->slot[slot]);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(ctl->sched_empty[slot]));
+      slot ^= 1;
+      if (!w.valid) break;
 
-        const TileRange un = key_tiles(w.pos0, w.pos0 + w.nrows, w.U);
-        TileRange hr[2];
-        int remaining[2];
+      const TileRange un = key_tiles(w.pos0, w.pos0 + w.nrows, w.U);
+      TileRange hr[2];
+      int remaining[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int lo = hh * kTileRows;
+        const int hi = w.nrows < lo + kTileRows ? w.nrows : lo + kTileRows;
+        hr[hh] = key_tiles(w.pos0 + lo, w.pos0 + (hi > lo ? hi : lo), w.U);
+        remaining[hh] = tile_count(hr[hh]);
+      }
+      const int n_u = tile_count(un);
+      if (!wait_all(bar(ctl->q_full), q_full_par)) break;
+      q_full_par ^= 1u;
+      ptx::tc_fence_after();
+
+      bool pend[2] = {false, false};
+      bool first[2] = {true, true};
+      int prev_vst = 0;
+      uint32_t prev_vph = 0;
+      // Step i, per half in turn: the P.V of the previous key tile (if that half used it), then
+      // the scores of key tile i (if that half needs it).  The tensor pipe therefore alternates
+      // [P.V_0, S_0], [P.V_1, S_1], and one half's SiLU overlaps the other half's MMAs.  The
+      // extra last step only drains the P.V.
+      for (int i = 0; i <= n_u; ++i) {
+        const bool last = (i == n_u);
+        int t = 0, kst = 0, vst = 0;
+        uint32_t kph = 0, vph = 0;
+        if (!last) {
+          t = tile_at(un, i);
+          kst = stage;
+          kph = kv_phase;
+          if (++stage == Cfg::kStages) { stage = 0; kv_phase ^= 1u; }
+          vst = stage;
+          vph = kv_phase;
+          if (++stage == Cfg::kStages) { stage = 0; kv_phase ^= 1u; }
+        }
+        bool k_waited = false, v_waited = false;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          const int lo = hh * kTileRows;
-          const int hi = w.nrows < lo + kTileRows ? w.nrows : lo + kTileRows;
-          hr[hh] = key_tiles(w.pos0 + lo, w.pos0 + (hi > lo ? hi : lo), w.U);
-          remaining[hh] = tile_count(hr[hh]);
-        }
-        const int n_u = tile_count(un);
-        if (!wait_bounded(bar(ctl->q_full), q_full_par, abort_flag, p.err)) break;
-        q_full_par ^= 1u;
-        ptx::tc_fence_after();
-
-        bool pend[2] = {false, false};
-        bool first[2] = {true, true};
-        int prev_vst = 0;
-        uint32_t prev_vph = 0;
-        // Step i, per half in turn: the P.V of the previous key tile (if that half used it), then
-        // the scores of key tile i (if that half needs it).  The tensor pipe therefore alternates
-        // [P.V_0, S_0], [P.V_1, S_1], and one half's SiLU overlaps the other half's MMAs.  The
-        // extra last step only drains the P.V.
-        for (int i = 0; i <= n_u; ++i) {
-          const bool last = (i == n_u);
-          int t = 0, kst = 0, vst = 0;
-          uint32_t kph = 0, vph = 0;
-          if (!last) {
-            t = tile_at(un, i);
-            kst = stage;
-            kph = kv_phase;
-            if (++stage == Cfg::kStages) { stage = 0; kv_phase ^= 1u; }
-            vst = stage;
-            vph = kv_phase;
-            if (++stage == Cfg::kStages) { stage = 0; kv_phase ^= 1u; }
-          }
-          bool k_waited = false, v_waited = false;
+          const uint32_t colS = hh ? Cfg::kColS1 : Cfg::kColS0;
+          if (pend[hh]) {
+            ok = wait_all(bar(ctl->p_full[hh]), p_full_par[hh]) &&
+                 (v_waited || wait_all(bar(ctl->kv_full[prev_vst]), prev_vph)) &&
+                 (!first[hh] || wait_all(bar(ctl->o_empty[hh]), o_empty_par[hh]));
+            if (!ok) break;
+            v_waited = true;
+            p_full_par[hh] ^= 1u;
+            if (first[hh]) o_empty_par[hh] ^= 1u;
+            ptx::tc_fence_after();
+            const uint64_t dv = dv0 + ((prev_vst * Cfg::kTileBytes) >> 4);
+            const uint32_t colO = hh ? Cfg::kColO1 : Cfg::kColO0;
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const uint32_t colS = hh ? Cfg::kColS1 : Cfg::kColS0;
-            if (pend[hh]) {
-              ok = wait_bounded(bar(ctl->p_full[hh]), p_full_par[hh], abort_flag, p.err) &&
-                   (v_waited || wait_bounded(bar(ctl->kv_full[prev_vst]), prev_vph, abort_flag, p.err)) &&
-                   (!first[hh] || wait_bounded(bar(ctl->o_empty[hh]), o_empty_par[hh], abort_flag, p.err));
-              if (!ok) break;
-              v_waited = true;
-              p_full_par[hh] ^= 1u;
-              if (first[hh]) o_empty_par[hh] ^= 1u;
+            for (int ks = 0; ks < kTileRows / 16; ++ks)
+              ptx::mma_ts_lead(lead, tmem + colO, tmem + colS + ks * 8, dv + ((ks * 16 * Cfg::kRowBytes) >> 4),
+                               Cfg::kIdescPV, (first[hh] && ks == 0) ? 0u : 1u);
+            first[hh] = false;
+            pend[hh] = false;
+            if (--remaining[hh] == 0) ptx::mma_commit_lead(lead, bar(ctl->o_full[hh]));
+          }
+          if (!last && tile_in(hr[hh], t)) {
+            if (!k_waited) {
+              if (!wait_all(bar(ctl->kv_full[kst]), kph)) { ok = false; break; }
               ptx::tc_fence_after();
-              const uint64_t dv = dv0 + ((prev_vst * Cfg::kTileBytes) >> 4);
-              const uint32_t colO = hh ? Cfg::kColO1 : Cfg::kColO0;
-#pragma unroll
-              for (int ks = 0; ks < kTileRows / 16; ++ks)
-                ptx::mma_ts(tmem + colO, tmem + colS + ks * 8, dv + ((ks * 16 * Cfg::kRowBytes) >> 4),
-                            Cfg::kIdescPV, (first[hh] && ks == 0) ? 0u : 1u);
-              first[hh] = false;
-              pend[hh] = false;
-              if (--remaining[hh] == 0) ptx::mma_commit(bar(ctl->o_full[hh]));
+              k_waited = true;
             }
-            if (!last && tile_in(hr[hh], t)) {
-              if (!k_waited) {
-                if (!wait_bounded(bar(ctl->kv_full[kst]), kph, abort_flag, p.err)) { ok = false; break; }
-                ptx::tc_fence_after();
-                k_waited = true;
-              }
-              const uint64_t dq = dq0 + ((hh * Cfg::kTileBytes) >> 4);
-              const uint64_t dk = dk0 + ((kst * Cfg::kTileBytes) >> 4);
+            const uint64_t dq = dq0 + ((hh * Cfg::kTileBytes) >> 4);
+            const uint64_t dk = dk0 + ((kst * Cfg::kTileBytes) >> 4);
 #pragma unroll
-              for (int ks = 0; ks < D / 16; ++ks) {
-                const uint32_t off =
-                    (ks / Cfg::kKStepsPerBlock) * Cfg::kBlockBytes + (ks % Cfg::kKStepsPerBlock) * 32;
-                ptx::mma_ss(tmem + colS, dq + (off >> 4), dk + (off >> 4), Cfg::kIdescQK, ks > 0 ? 1u : 0u);
-              }
-              ptx::mma_commit(bar(ctl->s_full[hh]));
-              pend[hh] = true;
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint32_t off =
+                  (ks / Cfg::kKStepsPerBlock) * Cfg::kBlockBytes + (ks % Cfg::kKStepsPerBlock) * 32;
+              ptx::mma_ss_lead(lead, tmem + colS, dq + (off >> 4), dk + (off >> 4), Cfg::kIdescQK,
+                               ks > 0 ? 1u : 0u);
             }
+            ptx::mma_commit_lead(lead, bar(ctl->s_full[hh]));
+            pend[hh] = true;
           }
-          if (!ok) break;
-          if (!last) ptx::mma_commit(bar(ctl->kv_empty[kst]));       // K_t: free after its S MMAs
-          if (i > 0) ptx::mma_commit(bar(ctl->kv_empty[prev_vst]));  // V_{t-1}: free after its P.V
-          if (i == n_u - 1) ptx::mma_commit(bar(ctl->q_empty));      // Q: free after the last S MMA
-          prev_vst = vst;
-          prev_vph = vph;
         }
+        if (!ok) break;
+        if (!last) ptx::mma_commit_lead(lead, bar(ctl->kv_empty[kst]));       // K_t: free after its S MMAs
+        if (i > 0) ptx::mma_commit_lead(lead, bar(ctl->kv_empty[prev_vst]));  // V_{t-1}: free after its P.V
+        if (i == n_u - 1) ptx::mma_commit_lead(lead, bar(ctl->q_empty));      // Q: free after the last S MMA
+        prev_vst = vst;
+        prev_vph = vph;
       }
-      // Every MMA this thread issued has completed once `drain` flips.
-      ptx::mma_commit(bar(ctl->drain));
-      drain_wait(bar(ctl->drain), 0u);
     }
+    // Every MMA lane 0 issued has completed once `drain` flips.
+    ptx::mma_commit_lead(lead, bar(ctl->drain));
+    drain_wait(bar(ctl->drain), 0u);
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ SiLU + epilogue
