@@ -33,6 +33,7 @@ EXPORTS = (
     "hstu_attn_fwd_noalloc",
     "hstu_attn_get_error",
     "hstu_attn_status_string",
+    "hstu_attn_selfcheck_wait_timeout",
 )
 
 
@@ -71,9 +72,10 @@ def load_library():
     lib.hstu_attn_fwd_noalloc.restype = ctypes.c_int
     lib.hstu_attn_get_error.argtypes = [vp]
     lib.hstu_attn_status_string.argtypes = [ctypes.c_int]
+    lib.hstu_attn_selfcheck_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.hstu_attn_status_string.restype = ctypes.c_char_p
     for name in ("hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_plan", "hstu_attn_fwd_planned",
-                 "hstu_attn_get_error"):
+                 "hstu_attn_get_error", "hstu_attn_selfcheck_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -257,3 +259,12 @@ def hstu_attn_get_error(device=None, stream=None):
 
 def hstu_attn_status_string(status):
     return load_library().hstu_attn_status_string(int(status)).decode()
+
+
+def hstu_attn_selfcheck_wait_timeout(limit_ns, device=None, stream=None):
+    """Launches the failure-path self-check: a bounded wait that must time out after limit_ns."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _raise_if(lib.hstu_attn_selfcheck_wait_timeout(int(limit_ns), _stream_ptr(stream, dev)),
+                  "hstu_attn_selfcheck_wait_timeout")

@@ -395,6 +395,14 @@ hstu_status_t hstu_attn_get_error(void* stream_ptr) {
   return HSTU_OK;
 }
 
+hstu_status_t hstu_attn_selfcheck_wait_timeout(uint64_t limit_ns, void* stream_ptr) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return HSTU_ERR_INVALID_ARGUMENT;
+  hstu::DeviceState* st = hstu::device_state();
+  if (!st) return HSTU_ERR_CUDA;
+  hstu::wait_timeout_selfcheck_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_ptr)>>>(st->err_word, limit_ns);
+  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
 const char* hstu_attn_status_string(hstu_status_t s) {
   switch (s) {
     case HSTU_OK: return "HSTU_OK";

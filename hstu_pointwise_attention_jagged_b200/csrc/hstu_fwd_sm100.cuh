@@ -107,14 +107,14 @@ __device__ __forceinline__ Work read_slot(const volatile int32_t* s) {
 
 // Slow path of wait_bounded: spins until the phase completes, the CTA aborts, or the time limit.
 __device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag,
-                                               unsigned* err) {
+                                               unsigned* err, uint64_t limit_ns) {
   const uint64_t t0 = ptx::globaltimer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (ptx::mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (ptx::globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicOr(err, kErrTimeout);
       return false;
@@ -125,9 +125,9 @@ __device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity, vo
 // Waits for phase `parity` of `bar`; false if the CTA is aborting or this wait timed out.  The
 // first test is inline: a call right after a burst of MMAs stalls the issuing warp.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag,
-                                             unsigned* err) {
+                                             unsigned* err, uint64_t limit_ns = kWaitLimitNs) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
-  return wait_bounded_slow(bar, parity, abort_flag, err);
+  return wait_bounded_slow(bar, parity, abort_flag, err, limit_ns);
 }
 
 // Abort-path drain: waits for phase `parity` of `bar` for at most kDrainLimitNs.
@@ -525,6 +525,22 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       atomicExch(p.done_counter, 0);
     }
   }
+}
+
+// Self-check of the failure path: one thread waits, through the bounded wait every role of the
+// attention kernel uses, on an mbarrier that nothing ever arrives on.  After limit_ns the wait
+// gives up, records kErrTimeout in the error word and raises the abort flag, and the kernel
+// returns normally: no trap, no hang, and the context stays usable.
+__global__ void wait_timeout_selfcheck_kernel(unsigned* err, uint64_t limit_ns) {
+  __shared__ uint64_t never;
+  __shared__ int32_t abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(ptx::smem_addr(&never), 1);
+    abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_bounded(ptx::smem_addr(&never), 0u, &abort_flag, err, limit_ns);
 }
 
 }  // namespace hstu

@@ -213,6 +213,18 @@ hstu_status_t hstu_attn_get_error(void* stream);
 /* Static, human-readable name of a status. */
 const char* hstu_attn_status_string(hstu_status_t s);
 
+/*
+ * hstu_attn_selfcheck_wait_timeout — exercises the failure-detection path on `stream`: one
+ * thread of a one-warp kernel waits, through the same bounded mbarrier wait every role of the
+ * attention kernel uses, on a barrier that nothing arrives on.  After limit_ns nanoseconds
+ * (1 .. 1e9) the wait gives up, sets the timeout bit of the device error word and the kernel
+ * returns; the next hstu_attn_get_error on the device reports HSTU_ERR_TIMEOUT and clears it.
+ * Nothing traps or hangs and the context stays usable.  Returns HSTU_ERR_INVALID_ARGUMENT for
+ * a limit outside the range, HSTU_ERR_CUDA if the launch fails, else HSTU_OK.  The pages have
+ * no counterpart: this is a test hook of the library's own failure handling.
+ */
+hstu_status_t hstu_attn_selfcheck_wait_timeout(uint64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

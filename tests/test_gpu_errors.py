@@ -73,3 +73,25 @@ def test_synchronous_argument_errors():
     with pytest.raises(binding.HstuError) as e:
         binding.hstu_attn_fwd(q, q, q, off, None, 1.0, 1.0, 16, out=q)
     assert e.value.status == 1
+
+
+def test_bounded_wait_times_out_and_reports():
+    """The bounded mbarrier wait every role of the attention kernel uses gives up on a barrier
+    that nothing arrives on: the kernel returns, the device reports HSTU_ERR_TIMEOUT once, and
+    the context still computes correct results afterwards (no trap, no hang)."""
+    assert binding.hstu_attn_get_error() == 0
+    binding.hstu_attn_selfcheck_wait_timeout(2_000_000)  # 2 ms
+    assert binding.hstu_attn_get_error() == 5  # HSTU_ERR_TIMEOUT
+    assert binding.hstu_attn_get_error() == 0  # cleared by the read
+    w = workloads.make_custom("after_timeout", [130, 40], [6, 3], 2, 64, 0.125, 140.0, seed=33)
+    out = binding.hstu_attn_fwd(dev_bf16(w.q), dev_bf16(w.k), dev_bf16(w.v), dev_i32(w.seq_offsets),
+                                dev_i32(w.num_targets), w.alpha, w.N, w.max_seq_len)
+    assert binding.hstu_attn_get_error() == 0
+    ref = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N)
+    assert_parity(to_f64(out), ref, what="after a timed-out self-check")
+
+
+def test_selfcheck_rejects_out_of_range_limits():
+    for bad in (0, 2_000_000_000):
+        with pytest.raises(binding.HstuError):
+            binding.hstu_attn_selfcheck_wait_timeout(bad)
