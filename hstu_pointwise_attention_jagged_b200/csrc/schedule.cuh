@@ -73,6 +73,7 @@ constexpr unsigned kErrTimeout = 2u;
 
 constexpr int kSchedThreads = 1024;
 constexpr int kMaxCostBins = 4096;
+constexpr int kCachedUsers = 256;  // batches up to this many users keep per-user values in shared memory
 
 struct SchedArgs {
   const int32_t* seq_offsets;  // [B+1]
@@ -117,6 +118,7 @@ __device__ __forceinline__ long long block_inclusive_scan(long long v, long long
 }
 
 // User owning block g: the last b with pair_start[b] <= g (users without blocks share a start).
+// pair_start may live in shared or global memory.
 __device__ __forceinline__ int owner_of(const int32_t* pair_start, int B, int g) {
   int lo = 0, hi = B;  // pair_start[lo] <= g < pair_start[hi]
   while (hi - lo > 1) {
@@ -136,6 +138,11 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
   __shared__ int hist[kMaxCostBins];
   __shared__ long long scan_scratch[32];
   __shared__ long long carry_q, carry_p;
+  // Per-user values of pass 1, kept on chip for passes 2 and 4 when the batch is small enough
+  // (their reads are then shared-memory latency instead of a chain of global loads).
+  __shared__ int s_L[kCachedUsers], s_U[kCachedUsers], s_c[kCachedUsers], s_q[kCachedUsers];
+  __shared__ int s_ps[kCachedUsers + 1];
+  const bool cached = a.B <= kCachedUsers;
   const int tid = threadIdx.x;
   const int nbins = a.nbins;
 
@@ -177,6 +184,14 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
       }
       a.q_start[b] = ok ? (int)start_q : -1;
       a.pair_start[b] = (int)start_p;
+      if (cached) {
+        const int o0 = a.seq_offsets[b], L = a.seq_offsets[b + 1] - o0;
+        s_L[b] = L;
+        s_U[b] = L - (a.num_targets ? a.num_targets[b] : 0);
+        s_c[b] = a.cached_len ? a.cached_len[b] : 0;
+        s_q[b] = ok ? (int)start_q : -1;
+        s_ps[b] = (int)start_p;
+      }
     }
     __syncthreads();
     if (tid == 0) {
@@ -188,20 +203,27 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
   const int npairs_total = (int)carry_p;
   if (tid == 0) {
     a.pair_start[a.B] = npairs_total;
+    if (cached) s_ps[a.B] = npairs_total;
     if (carry_q != a.total_q) atomicOr(a.err, kErrBadOffsets);
   }
   __syncthreads();
+  // Cost of block g (and its user), from shared memory when cached.
+  auto block_of = [&](int g, int& b, int& pr, int& cost) {
+    b = owner_of(cached ? s_ps : a.pair_start, a.B, g);
+    if ((cached ? s_q[b] : a.q_start[b]) < 0) return false;
+    const int L = cached ? s_L[b] : a.seq_offsets[b + 1] - a.seq_offsets[b];
+    const int U = cached ? s_U[b] : L - (a.num_targets ? a.num_targets[b] : 0);
+    const int c = cached ? s_c[b] : (a.cached_len ? a.cached_len[b] : 0);
+    pr = g - (cached ? s_ps[b] : a.pair_start[b]);
+    const int rows = (L - c) - pr * kPairRows;
+    cost = pair_cost(c + pr * kPairRows, rows < kPairRows ? rows : kPairRows, U);
+    return true;
+  };
 
   // Pass 2: cost histogram, one thread per block.
   for (int g = tid; g < npairs_total; g += kSchedThreads) {
-    const int b = owner_of(a.pair_start, a.B, g);
-    if (a.q_start[b] < 0) continue;
-    const int L = a.seq_offsets[b + 1] - a.seq_offsets[b];
-    const int U = L - (a.num_targets ? a.num_targets[b] : 0);
-    const int c = a.cached_len ? a.cached_len[b] : 0;
-    const int pr = g - a.pair_start[b];
-    const int rows = (L - c) - pr * kPairRows;
-    const int cost = pair_cost(c + pr * kPairRows, rows < kPairRows ? rows : kPairRows, U);
+    int b, pr, cost;
+    if (!block_of(g, b, pr, cost)) continue;
     atomicAdd(&hist[cost < nbins ? cost : nbins - 1], a.H);
   }
   __syncthreads();
@@ -234,14 +256,8 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
 
   // Pass 4: scatter the items into their bins, one thread per block.
   for (int g = tid; g < npairs_total; g += kSchedThreads) {
-    const int b = owner_of(a.pair_start, a.B, g);
-    if (a.q_start[b] < 0) continue;
-    const int L = a.seq_offsets[b + 1] - a.seq_offsets[b];
-    const int U = L - (a.num_targets ? a.num_targets[b] : 0);
-    const int c = a.cached_len ? a.cached_len[b] : 0;
-    const int pr = g - a.pair_start[b];
-    const int rows = (L - c) - pr * kPairRows;
-    const int cost = pair_cost(c + pr * kPairRows, rows < kPairRows ? rows : kPairRows, U);
+    int b, pr, cost;
+    if (!block_of(g, b, pr, cost)) continue;
     const int pos = atomicAdd(&hist[cost < nbins ? cost : nbins - 1], a.H);
     for (int h = 0; h < a.H; ++h)
       if (pos + h < a.max_items) a.items[pos + h] = make_int4(b, pr, h, cost);

@@ -260,19 +260,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Packed bf16 pair forms: tanh of both halves on the special-function unit, and a*b+c on both
-// halves with one rounding each (PTX tanh.approx.bf16x2, fma.rn.bf16x2).
-__device__ __forceinline__ uint32_t tanh_approx_bf16x2(uint32_t x) {
-  uint32_t y;
-  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-__device__ __forceinline__ uint32_t fma_bf16x2(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t y;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(y) : "r"(a), "r"(b), "r"(c));
-  return y;
-}
-
 // tanh on the special-function unit (PTX tanh.approx.f32).
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;

@@ -46,6 +46,9 @@ CASES = [
     ([1, 127, 128, 129, 0, 255, 256, 257, 1000], [0, 1, 2, 3, 0, 4, 0, 5, 300], None, 3),
     ([300, 513, 0, 700], [17, 0, 0, 129], [130, 0, 0, 200], 2),
     ([2048] * 8, [2048] * 8, None, 4),
+    # more users than the plan kernel keeps on chip: its global-memory path
+    (list(np.random.default_rng(41).integers(0, 700, 300)), list(np.random.default_rng(42).integers(0, 40, 300)),
+     None, 2),
 ]
 
 
