@@ -72,6 +72,32 @@ def test_stress_large_scores():
         assert_parity(got, ref, max_abs=1e-2 * np.abs(ref).max(), what="stress d=%d" % d)
 
 
+def test_many_small_users():
+    """1500 users of 0..60 history tokens and 0..8 candidates: thousands of work items, the plan
+    kernel's global-memory path (more users than it keeps on chip), every output compared."""
+    rng = np.random.default_rng(77)
+    uih = rng.integers(0, 61, 1500)
+    nt = rng.integers(0, 9, 1500)
+    w = workloads.make_custom("many", uih, nt, 2, 32, 1 / math.sqrt(32), float((uih + nt).max()), seed=78)
+    _full_compare(w, "1500 small users")
+
+
+def test_single_long_user():
+    """One user of 32768 tokens (30000 history + 2768 candidates), H=1, d=64: 128 query blocks of up to
+    235 key tiles each; sampled rows, including the last tiles and both sides of the history edge."""
+    w = workloads.make_custom("long1", [30000], [2768], 1, 64, 0.125, 32768.0, seed=79)
+    got_all = run_fwd(w)
+    users, local = sample_rows(w, per_user_random=96)
+    extra = np.array([29999 - 128, 29999, 30000, 32767 - 128, 32766], np.int32)
+    users = np.concatenate([users, np.zeros(len(extra), np.int32)])
+    local = np.concatenate([local, extra])
+    rows = query_row_index(w, users, local)
+    got = to_f64(got_all[torch.from_numpy(rows).cuda()])
+    ref = oracle.rows(w.q, w.k, w.v, w.seq_offsets, w.num_targets, None, w.alpha, w.N, users, local)
+    assert_parity(got, ref, what="single 32K-token user")
+    assert torch.isfinite(got_all.float()).all()
+
+
 @pytest.mark.parametrize("name", ["dlrmv3", "jagged", "long_history"])
 def test_full_size_sampled(name):
     """Full-size named workloads, one launch as the bench times it; sampled rows vs the oracle."""
