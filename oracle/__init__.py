@@ -38,8 +38,10 @@ class Oracle:
                                                i64, i64, f64, f64, f64p, i64p]
         lib.hstu_oracle_rows.argtypes = [f32p, f32p, f32p, i32p, i32p, i32p, i32, i32, i32, i64,
                                          i64, f64, f64, i32p, i32p, i64, f64p, i64p]
+        lib.hstu_oracle_rows_rab.argtypes = [f32p, f32p, f32p, i32p, i32p, i32p, f32p, i32, i32, i32,
+                                             i32, i64, i64, f64, f64, i32p, i32p, i64, f64p]
         for fn in (lib.hstu_oracle_fwd, lib.hstu_oracle_fwd_cached, lib.hstu_oracle_rows,
-                   lib.hstu_oracle_num_threads):
+                   lib.hstu_oracle_rows_rab, lib.hstu_oracle_num_threads):
             fn.restype = ctypes.c_int
         self.lib = lib
 
@@ -105,6 +107,39 @@ class Oracle:
         return (out, macs.value) if return_macs else out
 
 
+    def rows_rab(self, q, k, v, seq_offsets, num_targets, cached_len, rab, alpha, N, row_user, row_local):
+        """Selected rows of the relative-attention-bias variant; rab is the [H, R] bias table."""
+        q, k, v, rab = _f32(q), _f32(k), _f32(v), _f32(rab)
+        off = _i32(seq_offsets)
+        nt = None if num_targets is None else _i32(num_targets)
+        cl = None if cached_len is None else _i32(cached_len)
+        ru, rl = _i32(row_user), _i32(row_local)
+        total_q, H, d = q.shape
+        if rab.ndim != 2 or rab.shape[0] != H or rab.shape[1] < 1:
+            raise ValueError("oracle: rab must be [H, R] with R >= 1")
+        out = np.zeros((len(ru), H, d), dtype=np.float64)
+        rc = self.lib.hstu_oracle_rows_rab(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                           _ptr(v, ctypes.c_float), _ptr(off, ctypes.c_int32),
+                                           _ptr(nt, ctypes.c_int32), _ptr(cl, ctypes.c_int32),
+                                           _ptr(rab, ctypes.c_float), rab.shape[1], len(off) - 1, H, d,
+                                           k.shape[0], total_q, float(alpha), float(N),
+                                           _ptr(ru, ctypes.c_int32), _ptr(rl, ctypes.c_int32), len(ru),
+                                           _ptr(out, ctypes.c_double))
+        if rc != 0:
+            raise ValueError("oracle: inconsistent offsets, row selection or bias table")
+        return out
+
+    def fwd_rab(self, q, k, v, seq_offsets, num_targets, rab, alpha, N, cached_len=None):
+        """Every query row of the relative-attention-bias variant ([total_q, H, d]; with cached_len
+        the query rows are the new tokens, packed per user as in the library)."""
+        off = np.asarray(seq_offsets, np.int64)
+        L = np.diff(off)
+        c = np.zeros_like(L) if cached_len is None else np.asarray(cached_len, np.int64)
+        users = np.concatenate([np.full(max(int(L[b] - c[b]), 0), b) for b in range(len(L))] + [np.zeros(0)])
+        local = np.concatenate([np.arange(max(int(L[b] - c[b]), 0)) for b in range(len(L))] + [np.zeros(0)])
+        return self.rows_rab(q, k, v, seq_offsets, num_targets, cached_len, rab, alpha, N, users, local)
+
+
 def _f32(a):
     return np.ascontiguousarray(a, dtype=np.float32)
 
@@ -144,3 +179,11 @@ def fwd_cached(*args, **kwargs):
 
 def rows(*args, **kwargs):
     return default().rows(*args, **kwargs)
+
+
+def rows_rab(*args, **kwargs):
+    return default().rows_rab(*args, **kwargs)
+
+
+def fwd_rab(*args, **kwargs):
+    return default().fwd_rab(*args, **kwargs)

@@ -76,6 +76,32 @@ static int64_t one_row(const float* qrow, const float* kseg, const float* vseg, 
   return macs;
 }
 
+/*
+ * One output row of the relative-attention-bias variant.  The DLRMv3 review (section "model
+ * selection", time/position-encoding paragraph) prints the original HSTU attention, whose
+ * relative bias DLRMv3 drops, as Mask(SiLU(Q K^T) + bias) V.  Reading taken here, literally:
+ * each visible pair gets silu(alpha * s) plus a bias that depends only on the relative
+ * position i - j of query and key, read from the head's table rab_h[0 .. R-1] and clipped at
+ * its last entry; masked pairs contribute nothing.  Same arguments as one_row plus rab_h, R.
+ */
+static void one_row_rab(const float* qrow, const float* kseg, const float* vseg, int64_t stride,
+                        int32_t d, int32_t i, int32_t L, int32_t U, double alpha, double N,
+                        const float* rab_h, int32_t R, double* res) {
+  for (int32_t c = 0; c < d; ++c) res[c] = 0.0;
+  for (int32_t j = 0; j < L; ++j) {
+    if (!visible(i, j, U)) continue;
+    const float* krow = kseg + (int64_t)j * stride;
+    const float* vrow = vseg + (int64_t)j * stride;
+    double s = 0.0;
+    for (int32_t c = 0; c < d; ++c) s += (double)qrow[c] * (double)krow[c];
+    int32_t rel = i - j;
+    if (rel > R - 1) rel = R - 1;
+    double p = silu(alpha * s) + (double)rab_h[rel];
+    for (int32_t c = 0; c < d; ++c) res[c] += p * (double)vrow[c];
+  }
+  for (int32_t c = 0; c < d; ++c) res[c] /= N;
+}
+
 /* Checks one user's lengths; returns 0 if consistent. */
 static int user_ok(const int32_t* off, const int32_t* nt, const int32_t* cl, int32_t b,
                    int64_t total) {
@@ -221,4 +247,54 @@ int hstu_oracle_fwd_cached(const float* q_new, const float* k, const float* v,
   free(ru);
   free(rl);
   return rc;
+}
+
+/*
+ * Selected rows of the relative-attention-bias variant (one_row_rab); arguments as
+ * hstu_oracle_rows plus rab [H, R] (R >= 1).  Returns 0, or -1 on inconsistent input.
+ */
+int hstu_oracle_rows_rab(const float* q, const float* k, const float* v,
+                         const int32_t* seq_offsets, const int32_t* num_targets,
+                         const int32_t* cached_len, const float* rab, int32_t R, int32_t B,
+                         int32_t H, int32_t d, int64_t total_kv, int64_t total_q, double alpha,
+                         double N, const int32_t* row_user, const int32_t* row_local,
+                         int64_t nrows, double* out) {
+  if (B < 0 || H <= 0 || d <= 0 || R <= 0 || !rab || !(N != 0.0)) return -1;
+  if (seq_offsets[0] != 0 || seq_offsets[B] != total_kv) return -1;
+  int64_t* qstart = (int64_t*)malloc(sizeof(int64_t) * (size_t)(B + 1));
+  if (!qstart) return -1;
+  qstart[0] = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    if (user_ok(seq_offsets, num_targets, cached_len, b, total_kv)) { free(qstart); return -1; }
+    int32_t L = seq_offsets[b + 1] - seq_offsets[b];
+    int32_t c = cached_len ? cached_len[b] : 0;
+    qstart[b + 1] = qstart[b] + (L - c);
+  }
+  if (qstart[B] != total_q) { free(qstart); return -1; }
+  for (int64_t n = 0; n < nrows; ++n) {
+    int32_t b = row_user[n];
+    if (b < 0 || b >= B) { free(qstart); return -1; }
+    int32_t L = seq_offsets[b + 1] - seq_offsets[b];
+    int32_t c = cached_len ? cached_len[b] : 0;
+    if (row_local[n] < 0 || row_local[n] >= L - c) { free(qstart); return -1; }
+  }
+  const int64_t stride = (int64_t)H * d;
+  int64_t units = nrows * H;
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t u = 0; u < units; ++u) {
+    int64_t n = u / H;
+    int32_t h = (int32_t)(u % H);
+    int32_t b = row_user[n];
+    int32_t L = seq_offsets[b + 1] - seq_offsets[b];
+    int32_t T = num_targets ? num_targets[b] : 0;
+    int32_t c = cached_len ? cached_len[b] : 0;
+    int32_t r = row_local[n];
+    const float* qrow = q + (qstart[b] + r) * stride + (int64_t)h * d;
+    const float* kseg = k + (int64_t)seq_offsets[b] * stride + (int64_t)h * d;
+    const float* vseg = v + (int64_t)seq_offsets[b] * stride + (int64_t)h * d;
+    one_row_rab(qrow, kseg, vseg, stride, d, c + r, L, L - T, alpha, N, rab + (int64_t)h * R, R,
+                out + n * stride + (int64_t)h * d);
+  }
+  free(qstart);
+  return 0;
 }

@@ -240,7 +240,70 @@ def pin_flop_formula(o):
     assert 2 * per_matmul == 2 * (L * L * D // 2) + L * D, (macs, L, D)
 
 
-ALL_PINS = [pin_bruteforce_tiny, pin_bruteforce_random, pin_closed_form_counts, pin_zero_query, pin_single_token,
+def pin_rab_bruteforce(o):
+    """Relative-bias variant against the dense restatement, with a table shorter than the longest
+    distance (so clipping is exercised) and random entries of both signs."""
+    rng = np.random.default_rng(61)
+    q, k, v, off, nt = _rand_batch(rng, [23, 1, 17, 0, 30], [4, 1, 0, 0, 9], 2, 8)
+    rab = rng.normal(size=(2, 7)).astype(np.float32)
+    users, local = [], []
+    for b in range(len(off) - 1):
+        for r in range(int(off[b + 1] - off[b])):
+            users.append(b)
+            local.append(r)
+    got = o.rows_rab(q, k, v, off, nt, None, rab, 0.37, 11.0, users, local)
+    ref = bruteforce.attention_rab(q, k, v, off, nt, rab, 0.37, 11.0)
+    assert _rel(got, ref) <= 1e-12, _rel(got, ref)
+
+
+def pin_rab_constant_closed_form(o):
+    """A constant bias c adds c * (sum of the visible values) / N to every row: history rows the
+    prefix sum of v up to themselves, candidates the history sum plus their own v."""
+    rng = np.random.default_rng(62)
+    q, k, v, off, nt = _rand_batch(rng, [19, 33], [5, 3], 3, 4)
+    c = 0.625
+    rab = np.full((3, 4), c, np.float32)
+    users = [b for b in range(2) for _ in range(int(off[b + 1] - off[b]))]
+    local = [r for b in range(2) for r in range(int(off[b + 1] - off[b]))]
+    got = o.rows_rab(q, k, v, off, nt, None, rab, 0.5, 7.0, users, local)
+    base = o.fwd(q, k, v, off, nt, 0.5, 7.0)
+    vs = np.zeros_like(base)
+    for b in range(2):
+        s0, s1 = int(off[b]), int(off[b + 1])
+        U = (s1 - s0) - int(nt[b])
+        vv = v[s0:s1].astype(np.float64)
+        pref = np.cumsum(vv, axis=0)
+        for i in range(s1 - s0):
+            vs[s0 + i] = pref[i] if i < U else pref[U - 1] + vv[i]
+    assert _rel(got, base + c * vs / 7.0) <= 1e-12
+
+
+def pin_rab_zero_is_plain(o):
+    """A zero bias table reproduces the plain oracle exactly."""
+    rng = np.random.default_rng(63)
+    q, k, v, off, nt = _rand_batch(rng, [40, 9], [6, 2], 2, 16)
+    users = [b for b in range(2) for _ in range(int(off[b + 1] - off[b]))]
+    local = [r for b in range(2) for r in range(int(off[b + 1] - off[b]))]
+    got = o.rows_rab(q, k, v, off, nt, None, np.zeros((2, 3), np.float32), 0.2, 5.0, users, local)
+    assert np.array_equal(got, o.fwd(q, k, v, off, nt, 0.2, 5.0))
+
+
+def pin_rab_cached_equals_full(o):
+    """Cached rows of the bias variant equal the same positions of the full computation."""
+    rng = np.random.default_rng(64)
+    q, k, v, off, nt = _rand_batch(rng, [31, 12], [5, 4], 2, 8)
+    rab = rng.normal(size=(2, 9)).astype(np.float32)
+    cl = np.array([20, 7], np.int32)
+    users = [b for b in range(2) for _ in range(int(off[b + 1] - off[b] - cl[b]))]
+    local = [r for b in range(2) for r in range(int(off[b + 1] - off[b] - cl[b]))]
+    sel = np.concatenate([np.arange(off[b] + cl[b], off[b + 1]) for b in range(2)])
+    got = o.rows_rab(q[sel], k, v, off, nt, cl, rab, 0.3, 9.0, users, local)
+    full = bruteforce.attention_rab(q, k, v, off, nt, rab, 0.3, 9.0)[sel]
+    assert _rel(got, full) <= 1e-12
+
+
+ALL_PINS = [pin_rab_bruteforce, pin_rab_constant_closed_form, pin_rab_zero_is_plain, pin_rab_cached_equals_full,
+            pin_bruteforce_tiny, pin_bruteforce_random, pin_closed_form_counts, pin_zero_query, pin_single_token,
             pin_linear_regime, pin_negative_regime, pin_small_score_taylor, pin_causal_textbook,
             pin_history_ignores_candidates, pin_candidates_independent, pin_cached_equals_full,
             pin_linearity_and_scale, pin_flop_formula]

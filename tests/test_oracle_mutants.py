@@ -25,6 +25,10 @@ MUTANTS = {
     "off_by_one_history_length": ("static int64_t one_row(const float* qrow, const float* kseg, const float* vseg, int64_t stride,\n                       int32_t d, int32_t i, int32_t L, int32_t U, double alpha, double N,\n                       double* res) {\n  int64_t macs = 0;",
                                   "static int64_t one_row(const float* qrow, const float* kseg, const float* vseg, int64_t stride,\n                       int32_t d, int32_t i, int32_t L, int32_t U, double alpha, double N,\n                       double* res) {\n  int64_t macs = 0;\n  U = U + 1;"),
     "cached_position_ignores_prefix": ("d, c + r, L, L - T, alpha, N,", "d, r, L, L - T, alpha, N,"),
+    "rab_inside_silu": ("double p = silu(alpha * s) + (double)rab_h[rel];",
+                        "double p = silu(alpha * s + (double)rab_h[rel]);"),
+    "rab_ignores_position": ("int32_t rel = i - j;", "int32_t rel = 0;"),
+    "rab_clips_one_early": ("if (rel > R - 1) rel = R - 1;", "if (rel > R - 2) rel = R - 2;"),
 }
 
 
