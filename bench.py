@@ -38,6 +38,7 @@ METRIC = "jagged SiLU-attention TFLOP/s & target tokens/s, % of B200 BF16 TC pea
 WORKLOAD = "dlrmv3"
 FALLBACK_PEAK_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
+RAB_LEN = 4096  # relative-bias table entries per head for --variant rab
 
 
 # ------------------------------------------------------------------------------------ ranks
@@ -239,16 +240,26 @@ def run_ours(args, ranks):
     stream = torch.cuda.current_stream(dev)
     msl = w.max_seq_len
 
-    def step():
-        binding.hstu_attn_plan(off, nt, None, w.H, w.total, w.total, msl, plan=plan, stream=stream)
+    # The relative-attention-bias variant runs through its one-call entry point (plan included).
+    rab = None
+    if args.variant == "rab":
+        rab = torch.from_numpy(np.random.default_rng(rank_seed(5, ranks.rank)).normal(
+            scale=0.02, size=(w.H, RAB_LEN)).astype(np.float32)).to(dev)
 
     def attn():
-        binding.hstu_attn_fwd_planned(q, k, v, off, nt, None, w.alpha, w.N, plan, out=out, stream=stream)
+        if rab is None:
+            binding.hstu_attn_fwd_planned(q, k, v, off, nt, None, w.alpha, w.N, plan, out=out, stream=stream)
+        else:
+            binding.hstu_attn_fwd_rab(q, k, v, off, nt, rab, w.alpha, w.N, msl, out=out, stream=stream)
+
+    def step():
+        if rab is None:
+            binding.hstu_attn_plan(off, nt, None, w.H, w.total, w.total, msl, plan=plan, stream=stream)
+        attn()
 
     for _ in range(args.warmup):
         flush.zero_()
         step()
-        attn()
     torch.cuda.synchronize()
     status = binding.hstu_attn_get_error()
     if status != 0:
@@ -269,7 +280,6 @@ def run_ours(args, ranks):
             flush.zero_()
             ev[i][0].record(stream)
             step()
-            attn()
             ev[i][1].record(stream)
         for i in range(K):
             flush.zero_()
@@ -313,7 +323,10 @@ def run_ours(args, ranks):
             vd.copy_(v_h, non_blocking=True)
             od.copy_(off_h, non_blocking=True)
             nd.copy_(nt_h, non_blocking=True)
-            binding.hstu_attn_fwd(qd, kd, vd, od, nd, w.alpha, w.N, msl, out=outd, stream=streams[j])
+            if rab is None:
+                binding.hstu_attn_fwd(qd, kd, vd, od, nd, w.alpha, w.N, msl, out=outd, stream=streams[j])
+            else:
+                binding.hstu_attn_fwd_rab(qd, kd, vd, od, nd, rab, w.alpha, w.N, msl, out=outd, stream=streams[j])
             outs_h[j].copy_(outd, non_blocking=True)
 
     for i in range(4):
@@ -350,7 +363,8 @@ def run_ours(args, ranks):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1)/sqrt(d) bf16; DLRMv3 dataset unavailable)",
-        "config": workload_config(w, ranks.world),
+        "config": dict(workload_config(w, ranks.world), **({} if rab is None else {
+            "variant": "relative attention bias: silu(alpha*s) + rab[h, min(i-j, %d)]" % (RAB_LEN - 1)})),
         "target_tokens_per_s": round(job_targets / (ms_per_step * 1e-3), 1),
         "pct_of_peak": round(100.0 * value / ranks.world / peak, 2),
         "algorithmic_gflop_per_step": round(job_flops / 1e9, 3),
@@ -359,13 +373,18 @@ def run_ours(args, ranks):
                 "api": "hstu_attn_fwd (plan + attention) with pinned host buffers",
                 "pipelining": "2 streams, double-buffered device tensors: uploads, kernels and downloads of "
                               "neighbouring steps overlap; %d steps" % E},
-        "gpu_launches": 3 * K + 2 * E,
-        "roofline": {"bound": "tensor", "kernel": "hstu_fwd_kernel<128>", "achieved": round(achieved, 2),
+        "gpu_launches": (3 * K if rab is None else 4 * K) + 2 * E,
+        "roofline": {"bound": "tensor",
+                     "kernel": "hstu_fwd_kernel<128>" if rab is None else "hstu_fwd_kernel<128, rab> (+ plan kernel)",
+                     "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": args.traffic if args.traffic is not None else profiled_traffic(),
+                     "traffic": args.traffic if args.traffic is not None else (
+                         profiled_traffic() if rab is None else None),
                      "peak_source": peak_src,
                      "attn_ms_per_launch": round(attn_avg_ms, 5),
-                     "timing": "attention kernel alone, %d launches on one plan, L2 flushed before each" % K,
+                     "timing": ("attention kernel alone, %d launches on one plan, L2 flushed before each" % K
+                                if rab is None else
+                                "hstu_attn_fwd_rab calls (plan + attention), %d, L2 flushed before each" % K),
                      "flops_per_launch": int(flops)},
         "clocks": sampler.summary(),
     }
@@ -373,7 +392,11 @@ def run_ours(args, ranks):
         import oracle
         cores = oracle.num_threads()
         t0 = time.perf_counter()
-        _, macs = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N, return_macs=True)
+        if rab is None:
+            _, macs = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N, return_macs=True)
+        else:
+            oracle.fwd_rab(w.q, w.k, w.v, w.seq_offsets, w.num_targets, rab.cpu().numpy(), w.alpha, w.N)
+            macs = flops // 2
         dt = time.perf_counter() - t0
         line["cpu_baseline"] = {"value": 2 * macs / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                 "sample": "one full step: every row and head of the same batch (fp64 C oracle, "
@@ -428,6 +451,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ref-rows", type=int, default=0, help="rows per step of the reference arm (0: sized from K)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", choices=["plain", "rab"], default="plain",
+                    help="rab: the relative-attention-bias variant (a %d-entry table per head)" % RAB_LEN)
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of this kernel, if current")
     args = ap.parse_args(argv)

@@ -8,7 +8,7 @@ only new tokens against a cached K/V prefix.  The work happens in ``libhstu_attn
 ``include/hstu_attn.h``); :mod:`.binding` marshals torch tensors into it.  The binding's names
 are re-exported lazily so that :mod:`.workloads` and :mod:`.metrics` import without it.
 """
-_BINDING_NAMES = ("HstuError", "hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_plan_bytes", "hstu_attn_plan",
+_BINDING_NAMES = ("HstuError", "hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_fwd_rab", "hstu_attn_plan_bytes", "hstu_attn_plan",
                   "hstu_attn_fwd_planned", "hstu_attn_fwd_noalloc", "hstu_attn_get_error", "hstu_attn_status_string",
                   "hstu_attn_selfcheck_wait_timeout", "plan_contents",
                   "library_path", "load_library")

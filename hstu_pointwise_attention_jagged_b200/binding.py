@@ -27,6 +27,7 @@ STATUS = {
 EXPORTS = (
     "hstu_attn_fwd",
     "hstu_attn_fwd_cached",
+    "hstu_attn_fwd_rab",
     "hstu_attn_plan_bytes",
     "hstu_attn_plan",
     "hstu_attn_fwd_planned",
@@ -63,6 +64,8 @@ def load_library():
     lib.hstu_attn_fwd_cached.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, f32,
                                          vp, vp]
     i64 = ctypes.c_int64
+    lib.hstu_attn_fwd_rab.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, f32,
+                                      vp, vp]
     lib.hstu_attn_plan_bytes.argtypes = [i32, i32, i32]
     lib.hstu_attn_plan_bytes.restype = i64
     lib.hstu_attn_plan.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, i64, vp]
@@ -74,7 +77,7 @@ def load_library():
     lib.hstu_attn_status_string.argtypes = [ctypes.c_int]
     lib.hstu_attn_selfcheck_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.hstu_attn_status_string.restype = ctypes.c_char_p
-    for name in ("hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_plan", "hstu_attn_fwd_planned",
+    for name in ("hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_fwd_rab", "hstu_attn_plan", "hstu_attn_fwd_planned",
                  "hstu_attn_get_error", "hstu_attn_selfcheck_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -160,6 +163,38 @@ def hstu_attn_fwd_cached(q, k, v, seq_offsets, num_targets, cached_len, alpha, N
                                       _ptr(cached_len), B, H, d, total_kv, total_q, int(max_seq_len),
                                       float(alpha), float(N), _ptr(out), _stream_ptr(stream, q.device))
     _raise_if(st, "hstu_attn_fwd_cached")
+    return out
+
+
+def hstu_attn_fwd_rab(q, k, v, seq_offsets, num_targets, rab, alpha, N, max_seq_len, cached_len=None, out=None,
+                      stream=None):
+    """Relative-attention-bias variant: each visible pair gets silu(alpha*s) + rab[h, min(i-j, R-1)].
+    ``rab`` is a float32 [H, R] tensor on the same device; with ``cached_len`` the queries are the
+    new tokens only, as in :func:`hstu_attn_fwd_cached`.  Returns ``out``."""
+    lib = load_library()
+    _check_tokens("q", q)
+    total_q, H, d = q.shape
+    _check_tokens("k", k, H, d)
+    _check_tokens("v", v, H, d)
+    total_kv = k.shape[0]
+    if v.shape[0] != total_kv:
+        raise ValueError("k and v must have the same number of rows")
+    if rab.dtype != torch.float32 or rab.dim() != 2 or rab.shape[0] != H or not rab.is_contiguous() \
+            or rab.device != q.device:
+        raise TypeError("rab must be a contiguous float32 [H, R] tensor on %s" % q.device)
+    B = seq_offsets.numel() - 1
+    _check_index("seq_offsets", seq_offsets, B + 1, q.device, optional=False)
+    _check_index("num_targets", num_targets, B, q.device)
+    _check_index("cached_len", cached_len, B, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tokens("out", out, H, d)
+    with torch.cuda.device(q.device):
+        st = lib.hstu_attn_fwd_rab(_ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(num_targets),
+                                   _ptr(cached_len), _ptr(rab), int(rab.shape[1]), B, H, d, total_kv, total_q,
+                                   int(max_seq_len), float(alpha), float(N), _ptr(out),
+                                   _stream_ptr(stream, q.device))
+    _raise_if(st, "hstu_attn_fwd_rab")
     return out
 
 

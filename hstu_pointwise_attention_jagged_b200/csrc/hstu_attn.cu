@@ -42,8 +42,12 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 template <int D>
 cudaError_t set_kernel_attrs() {
-  return cudaFuncSetAttribute(hstu_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              FwdCfg<D>::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(hstu_fwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       FwdCfg<D>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(hstu_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FwdCfg<D>::kSmemBytes);
+  return e;
 }
 
 // One-time per-device set-up, run with that device current.
@@ -202,7 +206,7 @@ cudaError_t launch_plan(const int32_t* seq_offsets, const int32_t* num_targets, 
 // Launched as a programmatic dependent of the preceding kernel on the stream: its prologue
 // (barriers, TMEM allocation, tensor-map prefetch) overlaps the plan kernel, and the producer
 // waits for the preceding grid (griddepcontrol.wait) before its first global read.
-template <int D>
+template <int D, bool kRab>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                        int grid, cudaStream_t stream) {
   cudaLaunchConfig_t cfg;
@@ -216,14 +220,15 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, hstu_fwd_kernel<D>, tq, tk, tv, p);
+  return cudaLaunchKernelEx(&cfg, hstu_fwd_kernel<D, kRab>, tq, tk, tv, p);
 }
 
 // The attention kernel over a plan built for the same offsets.  Arguments already checked.
 hstu_status_t launch_attention(DeviceState* st, const void* q, const void* k, const void* v,
                                const int32_t* seq_offsets, const int32_t* num_targets, const int32_t* cached_len,
                                int32_t B, int32_t H, int32_t d, int32_t total_kv, int32_t total_q, float alpha,
-                               float N, void* plan, void* out, cudaStream_t stream) {
+                               float N, void* plan, void* out, cudaStream_t stream, const float* rab = nullptr,
+                               int32_t rab_len = 0) {
   if (!encoder()) return HSTU_ERR_CUDA;
   const int64_t row_elems = static_cast<int64_t>(H) * d;
   CUtensorMap tq, tk, tv;
@@ -243,6 +248,8 @@ hstu_status_t launch_attention(DeviceState* st, const void* q, const void* k, co
   p.work_counter = w.counter;
   p.done_counter = w.done;
   p.out = static_cast<__nv_bfloat16*>(out);
+  p.rab = rab;
+  p.rab_len = rab_len;
   p.H = H;
   p.half_alpha = 0.5f * alpha;
   p.inv_n = 1.0f / N;
@@ -250,9 +257,15 @@ hstu_status_t launch_attention(DeviceState* st, const void* q, const void* k, co
   const int64_t cap = capacity(B, H, total_q);
   const int grid = static_cast<int>(cap < st->num_sms ? cap : st->num_sms);
   cudaError_t e;
-  if (d == 128) e = launch_fwd<128>(tq, tk, tv, p, grid, stream);
-  else if (d == 64) e = launch_fwd<64>(tq, tk, tv, p, grid, stream);
-  else e = launch_fwd<32>(tq, tk, tv, p, grid, stream);
+  if (rab) {
+    if (d == 128) e = launch_fwd<128, true>(tq, tk, tv, p, grid, stream);
+    else if (d == 64) e = launch_fwd<64, true>(tq, tk, tv, p, grid, stream);
+    else e = launch_fwd<32, true>(tq, tk, tv, p, grid, stream);
+  } else {
+    if (d == 128) e = launch_fwd<128, false>(tq, tk, tv, p, grid, stream);
+    else if (d == 64) e = launch_fwd<64, false>(tq, tk, tv, p, grid, stream);
+    else e = launch_fwd<32, false>(tq, tk, tv, p, grid, stream);
+  }
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
@@ -260,7 +273,7 @@ hstu_status_t launch_attention(DeviceState* st, const void* q, const void* k, co
 hstu_status_t run(const void* q, const void* k, const void* v, const int32_t* seq_offsets,
                   const int32_t* num_targets, const int32_t* cached_len, int32_t B, int32_t H, int32_t d,
                   int32_t total_kv, int32_t total_q, int32_t max_seq_len, float alpha, float N, void* out,
-                  void* stream_ptr) {
+                  void* stream_ptr, const float* rab = nullptr, int32_t rab_len = 0) {
   hstu_status_t s = check_sizes(B, H, total_kv, total_q);
   if (s == HSTU_OK && max_seq_len < 0) s = HSTU_ERR_INVALID_ARGUMENT;
   if (s == HSTU_OK) s = check_tokens(q, k, v, seq_offsets, H, d, total_kv, total_q, alpha, N, out);
@@ -278,7 +291,7 @@ hstu_status_t run(const void* q, const void* k, const void* v, const int32_t* se
     s = HSTU_ERR_CUDA;
   if (s == HSTU_OK)
     s = launch_attention(st, q, k, v, seq_offsets, num_targets, cached_len, B, H, d, total_kv, total_q, alpha, N,
-                         plan, out, stream);
+                         plan, out, stream, rab, rab_len);
   if (cudaFreeAsync(plan, stream) != cudaSuccess && s == HSTU_OK) s = HSTU_ERR_CUDA;
   return s;
 }
@@ -340,6 +353,17 @@ hstu_status_t hstu_attn_fwd_cached(const void* q, const void* k, const void* v, 
                                    float N, void* out, void* stream) {
   return hstu::run(q, k, v, seq_offsets, num_targets, cached_len, B, H, d, total_kv, total_q, max_seq_len, alpha,
                    N, out, stream);
+}
+
+hstu_status_t hstu_attn_fwd_rab(const void* q, const void* k, const void* v, const int32_t* seq_offsets,
+                                const int32_t* num_targets, const int32_t* cached_len, const float* rab,
+                                int32_t rab_len, int32_t B, int32_t H, int32_t d, int32_t total_kv, int32_t total_q,
+                                int32_t max_seq_len, float alpha, float N, void* out, void* stream) {
+  if (rab_len < 1 || rab_len > (1 << 24)) return HSTU_ERR_INVALID_ARGUMENT;
+  if (!rab && total_q > 0 && B > 0) return HSTU_ERR_INVALID_ARGUMENT;
+  if (rab && (reinterpret_cast<uintptr_t>(rab) & 3u)) return HSTU_ERR_UNSUPPORTED;
+  return hstu::run(q, k, v, seq_offsets, num_targets, cached_len, B, H, d, total_kv, total_q, max_seq_len, alpha,
+                   N, out, stream, rab, rab_len);
 }
 
 int64_t hstu_attn_plan_bytes(int32_t B, int32_t H, int32_t total_q) {

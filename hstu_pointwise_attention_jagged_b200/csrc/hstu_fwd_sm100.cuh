@@ -69,6 +69,8 @@ struct FwdParams {
   int32_t* work_counter;
   int32_t* done_counter;
   __nv_bfloat16* out;
+  const float* rab;            // relative-bias variant: [H, rab_len] table; unused otherwise
+  int32_t rab_len;
   int32_t H;
   float half_alpha;
   float inv_n;
@@ -145,9 +147,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // SiLU + mask + bf16 pack of 32 score columns [32*chunk, 32*chunk+32) of this thread's row,
 // written as 16 packed columns [16*chunk, 16*chunk+16) of the same TMEM row.
 // lim/self are relative to the tile's first key: key column c is visible iff c < lim || c == self.
-template <int kChunk>
+// With kRab, a visible pair also gets rab_row[min(rel0 - c, rab_max)], its query-key distance
+// clipped to the last table entry (rel0 = query position - first key of the tile).
+template <int kChunk, bool kRab>
 __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t taddr_s, float half_alpha,
-                                           bool full, int lim, int self) {
+                                           bool full, int lim, int self, const float* rab_row, int rel0,
+                                           int rab_max) {
   uint32_t pk[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
@@ -155,6 +160,12 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t tad
     const float h1 = __uint_as_float(r[2 * e + 1]) * half_alpha;
     float p0 = fmaf(h0, ptx::tanh_approx(h0), h0);
     float p1 = fmaf(h1, ptx::tanh_approx(h1), h1);
+    if constexpr (kRab) {
+      // Distances of masked pairs can be negative: clamp so the read stays inside the table.
+      const int d0 = rel0 - (kChunk * 32 + 2 * e);
+      p0 += __ldg(rab_row + min(max(d0, 0), rab_max));
+      p1 += __ldg(rab_row + min(max(d0 - 1, 0), rab_max));
+    }
     if (!full) {
       const int c0 = kChunk * 32 + 2 * e;
       p0 = (c0 < lim || c0 == self) ? p0 : 0.0f;
@@ -165,7 +176,7 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t tad
   ptx::tmem_st16(taddr_s + kChunk * 16, pk);
 }
 
-template <int D>
+template <int D, bool kRab>
 __global__ void __launch_bounds__(kNumThreads, 1)
     hstu_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -452,6 +463,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       const int n = tile_count(r);
       const int i_pos = p0 + row;                      // this thread's query position
       const int lim_abs = (i_pos < w.U) ? i_pos + 1 : w.U;  // keys [0, lim_abs) visible, plus self
+      const float* rab_row = kRab ? p.rab + (size_t)w.h * p.rab_len : nullptr;
+      const int rab_max = kRab ? p.rab_len - 1 : 0;
       for (int k = 0; k < n; ++k) {
         const int j0 = tile_at(r, k) * kTileRows;
         ok = wait_bounded(bar(ctl->s_full[hh]), s_full_par, abort_flag, p.err);
@@ -462,20 +475,21 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const bool full = (j0 + kTileRows <= w.U) && (j0 + kTileRows <= p0 + 1);
         const int lim = lim_abs - j0;
         const int self = i_pos - j0;
+        const int rel0 = i_pos - j0;
         // 32-column chunks: the load of chunk c+1 is in flight while chunk c is computed.
         uint32_t ra[32], rb[32];
         ptx::tmem_ld32(taddr_s + 0, ra);
         ptx::tmem_ld_wait(ra);
         ptx::tmem_ld32(taddr_s + 32, rb);
-        silu_chunk<0>(ra, taddr_s, half_alpha, full, lim, self);
+        silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
         ptx::tmem_ld_wait(rb);
         ptx::tmem_ld32(taddr_s + 64, ra);
-        silu_chunk<1>(rb, taddr_s, half_alpha, full, lim, self);
+        silu_chunk<1, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
         ptx::tmem_ld_wait(ra);
         ptx::tmem_ld32(taddr_s + 96, rb);
-        silu_chunk<2>(ra, taddr_s, half_alpha, full, lim, self);
+        silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
         ptx::tmem_ld_wait(rb);
-        silu_chunk<3>(rb, taddr_s, half_alpha, full, lim, self);
+        silu_chunk<3, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();

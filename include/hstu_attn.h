@@ -124,6 +124,30 @@ hstu_status_t hstu_attn_fwd_cached(const void* q, const void* k, const void* v,
                                    void* out, void* stream);
 
 /*
+ * hstu_attn_fwd_rab — the relative-attention-bias variant that the DLRMv3 review (section
+ * "model selection", time/position-encoding paragraph) prints for the original HSTU,
+ * Mask(SiLU(Q K^T) + bias) V, and that DLRMv3 drops because it slows attention.  Reading taken:
+ * every visible pair (i, j) gets silu(alpha * <q_i, k_j>) + rab[h * rab_len + min(i - j,
+ * rab_len - 1)], a bias that depends only on the query-key distance, clipped at the table's
+ * last entry; masked pairs contribute nothing.  Positions i, j count from the start of the
+ * user's segment (cached prefix included), so the bias of a pair is the same in the full and
+ * the cached form.
+ *   rab      device float [H, rab_len], 4-byte aligned, read only; owned by the caller.
+ *   rab_len  1 .. 2^24 entries per head.
+ *   Other arguments as hstu_attn_fwd_cached; cached_len may be NULL (full sequences, q holds
+ *   every token).
+ * Errors: HSTU_ERR_INVALID_ARGUMENT for rab == NULL (with rows to compute) or rab_len out of
+ * range, HSTU_ERR_UNSUPPORTED for a misaligned table; otherwise as hstu_attn_fwd_cached.
+ */
+hstu_status_t hstu_attn_fwd_rab(const void* q, const void* k, const void* v,
+                                const int32_t* seq_offsets, const int32_t* num_targets,
+                                const int32_t* cached_len, const float* rab, int32_t rab_len,
+                                int32_t B, int32_t H, int32_t d,
+                                int32_t total_kv, int32_t total_q, int32_t max_seq_len,
+                                float alpha, float N,
+                                void* out, void* stream);
+
+/*
  * Two-step form.  hstu_attn_fwd / hstu_attn_fwd_cached are hstu_attn_plan followed by
  * hstu_attn_fwd_planned on a buffer the library takes from its own pool.  Callers that run the
  * attention several times over the same jagged structure (several layers, heads groups or

@@ -17,7 +17,8 @@ def declared_functions():
 
 
 def test_header_declares_the_entry_points():
-    assert declared_functions() == sorted(["hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_plan_bytes",
+    assert declared_functions() == sorted(["hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_fwd_rab",
+                                           "hstu_attn_plan_bytes",
                                            "hstu_attn_plan", "hstu_attn_fwd_planned", "hstu_attn_fwd_noalloc",
                                            "hstu_attn_get_error", "hstu_attn_status_string",
                                            "hstu_attn_selfcheck_wait_timeout"])
@@ -81,6 +82,12 @@ def test_host_validation_cached_and_planned(cuda_lib):
     st = cuda_lib.hstu_attn_fwd_planned(vp(4096), vp(4096), vp(4096), vp(4096), None, None, 1, 1, 64, 10, 10,
                                         1.0, 1.0, None, vp(1 << 20), None)
     assert st == 1
+    # the bias variant needs a table of 1 .. 2^24 entries per head
+    cuda_lib.hstu_attn_fwd_rab.argtypes = [vp] * 7 + [ctypes.c_int32] * 7 + [ctypes.c_float] * 2 + [vp, vp]
+    assert cuda_lib.hstu_attn_fwd_rab(vp(4096), vp(4096), vp(4096), vp(4096), None, None, None, 16, 1, 1, 64, 10, 10,
+                                      10, 1.0, 1.0, vp(1 << 20), None) == 1
+    assert cuda_lib.hstu_attn_fwd_rab(vp(4096), vp(4096), vp(4096), vp(4096), None, None, vp(4096), 0, 1, 1, 64, 10,
+                                      10, 10, 1.0, 1.0, vp(1 << 20), None) == 1
     # the failure-path self-check takes limits of 1 ns .. 1 s only
     cuda_lib.hstu_attn_selfcheck_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     assert cuda_lib.hstu_attn_selfcheck_wait_timeout(0, None) == 1
