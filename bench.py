@@ -375,7 +375,7 @@ def run_ours(args, ranks):
                               "neighbouring steps overlap; %d steps" % E},
         "gpu_launches": (3 * K if rab is None else 4 * K) + 2 * E,
         "roofline": {"bound": "tensor",
-                     "kernel": "hstu_fwd_kernel<128>" if rab is None else "hstu_fwd_kernel<128, rab> (+ plan kernel)",
+                     "kernel": "hstu_fwd_kernel<128, 0>" if rab is None else "hstu_fwd_kernel<128, rab> (+ plan kernel)",
                      "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": args.traffic if args.traffic is not None else (
