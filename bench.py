@@ -404,6 +404,130 @@ def run_ours(args, ranks):
     return line
 
 
+def run_proj(args, ranks):
+    """The HSTU layer's two dense projections around the attention of the DLRMv3-shaped batch
+    (L = 32768 token rows, D = H*d = 512): [L, D] x [D, 4D] and [L, 3D] x [3D, D], the 4*L*D^2 and
+    3*L*D^2 terms of the review's per-layer FLOP formula, through hstu_attn_gemm_bf16.  cuBLAS
+    (torch.matmul) is timed on the same shapes for context only."""
+    import torch
+    from hstu_pointwise_attention_jagged_b200 import binding, workloads
+
+    dev = torch.device("cuda", ranks.local_rank)
+    torch.cuda.set_device(dev)
+    binding.load_library()
+    w = workloads.make(WORKLOAD, seed=rank_seed(1, ranks.rank))
+    L, D = w.total, w.H * w.d
+    shapes = [(L, 4 * D, D), (L, D, 3 * D)]
+    rng = np.random.default_rng(rank_seed(11, ranks.rank))
+
+    def bf16(x):
+        return torch.from_numpy(workloads.bf16_bits(workloads.round_bf16(x.astype(np.float32))).view(np.int16)).view(
+            torch.bfloat16)
+
+    host = [(bf16(rng.standard_normal((M, K))).pin_memory(), bf16(rng.standard_normal((N, K)) / np.sqrt(K)).pin_memory())
+            for M, N, K in shapes]
+    devm = [(a.to(dev), b.to(dev)) for a, b in host]
+    outs = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for M, N, K in shapes]
+    flops = sum(2 * M * N * K for M, N, K in shapes)
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for (a, b), o in zip(devm, outs):
+            binding.hstu_attn_gemm_bf16(a, b, out=o, stream=stream)
+
+    def step_cublas():
+        for (a, b), o in zip(devm, outs):
+            torch.matmul(a, b.t(), out=o)
+
+    def timed(fn, K):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            fn()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+        step_cublas()
+    torch.cuda.synchronize()
+    if binding.hstu_attn_get_error() != 0:
+        raise RuntimeError("warm-up reported an error")
+    K = args.steps
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    ranks.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        total_ms = ranks.max(timed(step, K), dev)
+        cublas_ms = ranks.max(timed(step_cublas, K), dev)
+        ranks.barrier()
+    if binding.hstu_attn_get_error() != 0:
+        raise RuntimeError("timed steps reported an error")
+    ms = total_ms / K
+    job_flops = ranks.sum(flops, dev)
+    value = job_flops / (ms * 1e-3) / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    peak, peak_src = measured_peak()
+
+    # End to end: inputs from pinned host memory, outputs back, every step.
+    outs_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    E = max(4, min(args.steps, 50))
+    h2d = sum(a.numel() * 2 + b.numel() * 2 for a, b in host)
+    d2h = sum(o.numel() * 2 for o in outs)
+
+    def e2e_step():
+        for (ah, bh), (a, b), o, oh in zip(host, devm, outs, outs_h):
+            a.copy_(ah, non_blocking=True)
+            b.copy_(bh, non_blocking=True)
+            binding.hstu_attn_gemm_bf16(a, b, out=o, stream=stream)
+            oh.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ranks.max(e0.elapsed_time(e1), dev) / E
+
+    line = {
+        "metric": "HSTU layer projection GEMMs TFLOP/s (input [L,D]x[D,4D] and output [L,3D]x[3D,D])",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ranks.world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) activations, N(0,1/K) weights, bf16)",
+        "config": {"workload": "dlrmv3 layer projections: L=%d, D=%d; shapes (M,N,K) %s" % (L, D, shapes),
+                   "parallelism": "dp%d (token rows sharded, no collective)" % ranks.world,
+                   "l2": "flushed before every timed step (256 MiB write)"},
+        "e2e": {"value": round(job_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 2 * K + 2 * E,
+        "roofline": {"bound": "tensor", "kernel": "gemm_bf16_kernel", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None, "peak_source": peak_src,
+                     "flops_per_step": int(flops)},
+        "cublas_same_shapes": {"value": round(flops / (cublas_ms / K * 1e-3) / 1e12, 2), "unit": "TFLOP/s"},
+        "clocks": sampler.summary(),
+    }
+    if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline:
+        import oracle
+        rows = 2048
+        t0 = time.perf_counter()
+        for (ah, bh), (M, N, Kd) in zip(host, shapes):
+            oracle.linear(ah[:rows].float().numpy(), bh.float().numpy())
+        dt = time.perf_counter() - t0
+        sample_flops = sum(2 * rows * N * Kd for M, N, Kd in shapes)
+        line["cpu_baseline"] = {"value": sample_flops / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                                "kind": "oracle", "sample": "the first %d rows of both projections (fp64 numpy "
+                                                            "matmul), %.2f s" % (rows, dt)}
+    return line
+
+
 def run_reference(args, world):
     """The fp64 oracle on the host cores, rank 0 only: each step a bounded row sample, sized so that
     warm-up plus K steps stay near a minute of CPU work."""
@@ -451,8 +575,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ref-rows", type=int, default=0, help="rows per step of the reference arm (0: sized from K)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", choices=["plain", "rab"], default="plain",
-                    help="rab: the relative-attention-bias variant (a %d-entry table per head)" % RAB_LEN)
+    ap.add_argument("--variant", choices=["plain", "rab", "proj"], default="plain",
+                    help="rab: the relative-attention-bias variant (a %d-entry table per head); proj: the layer's "
+                         "projection GEMMs" % RAB_LEN)
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of this kernel, if current")
     args = ap.parse_args(argv)
@@ -468,7 +593,7 @@ def main(argv=None):
         return 0
     ranks = Ranks(backend="nccl")
     try:
-        line = run_ours(args, ranks)
+        line = run_proj(args, ranks) if args.variant == "proj" else run_ours(args, ranks)
     finally:
         ranks.close()
     if ranks.rank == 0:

@@ -35,6 +35,7 @@ EXPORTS = (
     "hstu_attn_get_error",
     "hstu_attn_status_string",
     "hstu_attn_selfcheck_wait_timeout",
+    "hstu_attn_gemm_bf16",
 )
 
 
@@ -76,9 +77,10 @@ def load_library():
     lib.hstu_attn_get_error.argtypes = [vp]
     lib.hstu_attn_status_string.argtypes = [ctypes.c_int]
     lib.hstu_attn_selfcheck_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.hstu_attn_gemm_bf16.argtypes = [vp, vp, vp, i32, i32, i32, vp]
     lib.hstu_attn_status_string.restype = ctypes.c_char_p
     for name in ("hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_fwd_rab", "hstu_attn_plan", "hstu_attn_fwd_planned",
-                 "hstu_attn_get_error", "hstu_attn_selfcheck_wait_timeout"):
+                 "hstu_attn_get_error", "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -303,3 +305,23 @@ def hstu_attn_selfcheck_wait_timeout(limit_ns, device=None, stream=None):
     with torch.cuda.device(dev):
         _raise_if(lib.hstu_attn_selfcheck_wait_timeout(int(limit_ns), _stream_ptr(stream, dev)),
                   "hstu_attn_selfcheck_wait_timeout")
+
+
+def hstu_attn_gemm_bf16(a, w, out=None, stream=None):
+    """C = A · Wᵀ (bf16 [M, K] · bf16 [N, K]ᵀ -> bf16 [M, N]) on the tensor cores; returns ``out``."""
+    lib = load_library()
+    for name, t in (("a", a), ("w", w)):
+        if t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_contiguous() or not t.is_cuda:
+            raise TypeError("%s must be a contiguous bf16 CUDA matrix" % name)
+    M, K = a.shape
+    N = w.shape[0]
+    if w.shape[1] != K or w.device != a.device:
+        raise ValueError("w must be [N, K] on the same device as a")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != (M, N) or not out.is_contiguous():
+        raise TypeError("out must be a contiguous bf16 [M, N] tensor")
+    with torch.cuda.device(a.device):
+        st = lib.hstu_attn_gemm_bf16(_ptr(a), _ptr(w), _ptr(out), M, N, K, _stream_ptr(stream, a.device))
+    _raise_if(st, "hstu_attn_gemm_bf16")
+    return out

@@ -1,0 +1,213 @@
+// gemm_sm100.cuh — bf16 GEMM C = A · Wᵀ with fp32 accumulation on the sm_100a tensor cores.
+//
+// The HSTU layer around the attention (DLRMv3 review, section "model selection", FLOP-formula
+// paragraph: per layer 2·(L²·D/2 + 4·L·D² + 3·L·D²) flops) spends its non-attention work in dense
+// projections of the L token rows.  This kernel computes one such projection: A is [M, K] (token
+// rows), W is [N, K] (the weight in the out-features × in-features layout of a linear layer), C is
+// [M, N]; all bf16, row-major.
+//
+// Persistent and warp-specialised, one CTA per SM:
+//   warp 0       TMA producer: 128×64 tiles of A and 256×64 tiles of W into a 4-stage ring
+//                (128-byte swizzle, K-major, zero fill past the edges);
+//   warp 1       MMA issuer: per 64-deep k block four tcgen05.mma 128×256×16 (each instruction
+//                carries 128 clocks of tensor work, so the issuing thread has slack for its
+//                waits and commits) into one of two TMEM accumulators of 256 columns;
+//   warps 2..5   epilogue: TMEM -> registers -> bf16 -> row- and column-predicated 16-byte stores,
+//                overlapping the next tile's main loop on the other accumulator.
+// Output tiles are visited in M-fastest order, so CTAs working at the same time share W tiles in
+// L2.  Every wait is bounded; a timeout sets the error word and the kernel drains and returns.
+#pragma once
+
+#include "hstu_fwd_sm100.cuh"
+
+namespace hstu {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBN = 256;
+constexpr int kGemmBK = 64;  // one 128-byte swizzle atom of bf16
+constexpr int kGemmStages = 4;
+constexpr int kGemmThreads = 192;
+
+struct GemmCfg {
+  static constexpr int kABytes = kGemmBM * kGemmBK * 2;  // 16 KB
+  static constexpr int kBBytes = kGemmBN * kGemmBK * 2;  // 32 KB
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kSmemBytes = 1024 + kGemmStages * kStageBytes + 1024;
+  static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(kGemmBM, kGemmBN, false);
+};
+
+struct GemmCtl {
+  uint64_t full[kGemmStages], empty[kGemmStages];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int32_t abort_flag;
+};
+
+struct GemmParams {
+  __nv_bfloat16* c;
+  int32_t M, N, K;
+  int32_t tiles_m, tiles_n;
+  unsigned* err;
+};
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
+                     const GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw_addr = ptx::smem_addr(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  const uint32_t sbase = ptx::smem_addr(smem);
+  auto* ctl = reinterpret_cast<GemmCtl*>(smem + kGemmStages * GemmCfg::kStageBytes);
+  volatile int32_t* abort_flag = &ctl->abort_flag;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  auto bar = [](const uint64_t& b) { return ptx::smem_addr(&b); };
+  auto sA = [&](int s) { return sbase + s * GemmCfg::kStageBytes; };
+  auto sB = [&](int s) { return sbase + s * GemmCfg::kStageBytes + GemmCfg::kABytes; };
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < kGemmStages; ++s) {
+      ptx::mbar_init(bar(ctl->full[s]), 1);
+      ptx::mbar_init(bar(ctl->empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(bar(ctl->acc_full[a]), 1);
+      ptx::mbar_init(bar(ctl->acc_empty[a]), 4);  // one arrival per epilogue warp
+    }
+    ptx::mbar_init(bar(ctl->drain), 1);
+    ctl->abort_flag = 0;
+    ptx::fence_mbarrier_init();
+    ptx::prefetch_tmap(&tm_a);
+    ptx::prefetch_tmap(&tm_w);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(&ctl->tmem_base), 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  const int ntiles = p.tiles_m * p.tiles_n;
+  const int kblocks = (p.K + kGemmBK - 1) / kGemmBK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % p.tiles_m) * kGemmBM;
+        const int n0 = (tile / p.tiles_m) * kGemmBN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!wait_bounded(bar(ctl->empty[stage]), phase ^ 1u, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar(ctl->full[stage]);
+          ptx::mbar_arrive_expect_tx(fb, GemmCfg::kStageBytes);
+          ptx::tma_load_2d(sA(stage), &tm_a, fb, kb * kGemmBK, m0);
+          ptx::tma_load_2d(sB(stage), &tm_w, fb, kb * kGemmBK, n0);
+          ++issued;
+          if (++stage == kGemmStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (*abort_flag) {
+        // Let every copy this CTA started land before its shared memory is released.
+        for (int k = 1; k <= kGemmStages && k <= issued; ++k) {
+          const int pos = issued - k;
+          drain_wait(bar(ctl->full[pos % kGemmStages]), (uint32_t)((pos / kGemmStages) & 1));
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    const uint32_t lead = (lane == 0) ? 1u : 0u;
+    auto wait_all = [&](uint32_t b, uint32_t par) {
+      return __all_sync(0xffffffffu, wait_bounded(b, par, abort_flag, p.err));
+    };
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t acc_empty_par[2] = {1u, 1u};
+    int acc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      ok = wait_all(bar(ctl->acc_empty[acc]), acc_empty_par[acc]);
+      if (!ok) break;
+      acc_empty_par[acc] ^= 1u;
+      ptx::tc_fence_after();
+      const uint32_t dacc = tmem + acc * kGemmBN;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        ok = wait_all(bar(ctl->full[stage]), phase);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const uint64_t da = ptx::smem_desc(sA(stage), 16, 1024, 2);
+        const uint64_t db = ptx::smem_desc(sB(stage), 16, 1024, 2);
+#pragma unroll
+        for (int ks = 0; ks < kGemmBK / 16; ++ks)  // +32 bytes along the swizzled row per k step
+          ptx::mma_ss_lead(lead, dacc, da + ks * 2, db + ks * 2, GemmCfg::kIdesc, (kb | ks) ? 1u : 0u);
+        ptx::mma_commit_lead(lead, bar(ctl->empty[stage]));
+        if (++stage == kGemmStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      ptx::mma_commit_lead(lead, bar(ctl->acc_full[acc]));
+      acc ^= 1;
+    }
+    ptx::mma_commit_lead(lead, bar(ctl->drain));
+    drain_wait(bar(ctl->drain), 0u);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2..5)
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    uint32_t acc_full_par[2] = {0u, 0u};
+    int acc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+      ok = __all_sync(0xffffffffu, wait_bounded(bar(ctl->acc_full[acc]), acc_full_par[acc], abort_flag, p.err));
+      if (!ok) break;
+      acc_full_par[acc] ^= 1u;
+      ptx::tc_fence_after();
+      const int m = (tile % p.tiles_m) * kGemmBM + row;
+      const int n0 = (tile / p.tiles_m) * kGemmBN;
+      __nv_bfloat16* dst = p.c + (size_t)(m < p.M ? m : 0) * p.N + n0;
+#pragma unroll 1
+      for (int c = 0; c < kGemmBN / 32; ++c) {
+        uint32_t r[32];
+        ptx::tmem_ld32(tmem + lane_off + acc * kGemmBN + c * 32, r);
+        ptx::tmem_ld_wait(r);
+        if (m < p.M) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int n = n0 + c * 32 + q4 * 8;
+            if (n < p.N) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
+              v.y = pack_bf16x2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
+              v.z = pack_bf16x2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
+              v.w = pack_bf16x2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
+              *reinterpret_cast<uint4*>(dst + c * 32 + q4 * 8) = v;
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(ctl->acc_empty[acc]));
+      acc ^= 1;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 1) ptx::tmem_dealloc(tmem, 512);
+}
+
+}  // namespace hstu

@@ -17,6 +17,7 @@
 
 #include "hstu_attn.h"
 #include "hstu_fwd_sm100.cuh"
+#include "gemm_sm100.cuh"
 #include "schedule.cuh"
 
 namespace hstu {
@@ -71,6 +72,8 @@ void init_device(DeviceState& st, int dev) {
   if (e == cudaSuccess) e = set_kernel_attrs<32>();
   if (e == cudaSuccess) e = set_kernel_attrs<64>();
   if (e == cudaSuccess) e = set_kernel_attrs<128>();
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg::kSmemBytes);
   st.init_err = e;
 }
 
@@ -103,6 +106,18 @@ bool encode_rows(CUtensorMap* map, const void* base, int64_t rows, int64_t row_e
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// A row-major bf16 [rows, cols] matrix read in boxes of box_rows x 64 columns, 128-byte swizzle.
+bool encode_matrix(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2u};
+  cuuint32_t box[2] = {64u, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -417,6 +432,37 @@ hstu_status_t hstu_attn_get_error(void* stream_ptr) {
   if (word & hstu::kErrTimeout) return HSTU_ERR_TIMEOUT;
   if (word & hstu::kErrBadOffsets) return HSTU_ERR_BAD_OFFSETS;
   return HSTU_OK;
+}
+
+hstu_status_t hstu_attn_gemm_bf16(const void* a, const void* w, void* c, int32_t M, int32_t N, int32_t K,
+                             void* stream_ptr) {
+  if (M < 0 || N < 0 || K <= 0) return HSTU_ERR_INVALID_ARGUMENT;
+  if (M == 0 || N == 0) return HSTU_OK;
+  if (!a || !w || !c) return HSTU_ERR_INVALID_ARGUMENT;
+  if ((K % 8) != 0 || (N % 8) != 0) return HSTU_ERR_UNSUPPORTED;  // 16-byte rows for TMA and stores
+  if (!hstu::aligned16(a) || !hstu::aligned16(w) || !hstu::aligned16(c)) return HSTU_ERR_UNSUPPORTED;
+  const size_t ca = static_cast<size_t>(M) * K * 2, cw = static_cast<size_t>(N) * K * 2,
+               cc = static_cast<size_t>(M) * N * 2;
+  if (hstu::overlaps(c, cc, a, ca) || hstu::overlaps(c, cc, w, cw)) return HSTU_ERR_INVALID_ARGUMENT;
+  hstu::DeviceState* st = hstu::device_state();
+  if (!st || !hstu::encoder()) return HSTU_ERR_CUDA;
+  CUtensorMap ta, tw;
+  if (!hstu::encode_matrix(&ta, a, M, K, hstu::kGemmBM) || !hstu::encode_matrix(&tw, w, N, K, hstu::kGemmBN))
+    return HSTU_ERR_CUDA;
+  hstu::GemmParams p;
+  p.c = static_cast<__nv_bfloat16*>(c);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.tiles_m = (M + hstu::kGemmBM - 1) / hstu::kGemmBM;
+  p.tiles_n = (N + hstu::kGemmBN - 1) / hstu::kGemmBN;
+  p.err = st->err_word;
+  const int64_t ntiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+  if (ntiles > INT_MAX) return HSTU_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(ntiles < st->num_sms ? ntiles : st->num_sms);
+  hstu::gemm_bf16_kernel<<<grid, hstu::kGemmThreads, hstu::GemmCfg::kSmemBytes,
+                           static_cast<cudaStream_t>(stream_ptr)>>>(ta, tw, p);
+  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
 hstu_status_t hstu_attn_selfcheck_wait_timeout(uint64_t limit_ns, void* stream_ptr) {

@@ -238,6 +238,22 @@ hstu_status_t hstu_attn_get_error(void* stream);
 const char* hstu_attn_status_string(hstu_status_t s);
 
 /*
+ * hstu_attn_gemm_bf16 — C = A · Wᵀ on the tensor cores: A bf16 [M, K], W bf16 [N, K] (a linear
+ * layer's weight, out-features × in-features), C bf16 [M, N], all row-major on the device;
+ * products accumulate in fp32 and are rounded to bf16 once.  These are the dense projections
+ * of the HSTU layer around the attention, whose flops the DLRMv3 review counts as 4·L·D² and
+ * 3·L·D² per layer (section "model selection", FLOP-formula paragraph); the pages do not give
+ * the layer's other steps.
+ *   M, N >= 0 (M or N == 0: nothing is done), K >= 1; K and N multiples of 8 (16-byte rows);
+ *   pointers 16-byte aligned; C must not overlap A or W.  Asynchronous on `stream`.
+ * Errors: HSTU_ERR_INVALID_ARGUMENT (NULL pointers, negative sizes, overlap),
+ * HSTU_ERR_UNSUPPORTED (alignment, K or N not a multiple of 8), HSTU_ERR_CUDA (launch); a
+ * device-side timeout is reported by hstu_attn_get_error.
+ */
+hstu_status_t hstu_attn_gemm_bf16(const void* a, const void* w, void* c, int32_t M, int32_t N, int32_t K,
+                             void* stream);
+
+/*
  * hstu_attn_selfcheck_wait_timeout — exercises the failure-detection path on `stream`: one
  * thread of a one-warp kernel waits, through the same bounded mbarrier wait every role of the
  * attention kernel uses, on a barrier that nothing arrives on.  After limit_ns nanoseconds

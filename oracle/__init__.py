@@ -187,3 +187,9 @@ def rows_rab(*args, **kwargs):
 
 def fwd_rab(*args, **kwargs):
     return default().fwd_rab(*args, **kwargs)
+
+
+def linear(a, w):
+    """C = A · Wᵀ in fp64 (A [M, K], W [N, K]): the dense projections of the HSTU layer whose flops
+    the DLRMv3 review counts as 4·L·D² and 3·L·D² per layer.  A matrix product is the definition."""
+    return np.asarray(a, np.float64) @ np.asarray(w, np.float64).T

@@ -21,7 +21,7 @@ def test_header_declares_the_entry_points():
                                            "hstu_attn_plan_bytes",
                                            "hstu_attn_plan", "hstu_attn_fwd_planned", "hstu_attn_fwd_noalloc",
                                            "hstu_attn_get_error", "hstu_attn_status_string",
-                                           "hstu_attn_selfcheck_wait_timeout"])
+                                           "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16"])
 
 
 def test_library_exports_every_declared_symbol(cuda_lib):
@@ -88,6 +88,15 @@ def test_host_validation_cached_and_planned(cuda_lib):
                                       10, 1.0, 1.0, vp(1 << 20), None) == 1
     assert cuda_lib.hstu_attn_fwd_rab(vp(4096), vp(4096), vp(4096), vp(4096), None, None, vp(4096), 0, 1, 1, 64, 10,
                                       10, 10, 1.0, 1.0, vp(1 << 20), None) == 1
+    # the GEMM: K and N multiples of 8, aligned pointers, no overlap of C with A or W
+    g = cuda_lib.hstu_attn_gemm_bf16
+    g.argtypes = [vp, vp, vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp]
+    assert g(vp(4096), vp(1 << 22), vp(1 << 24), 16, 16, 12, None) == 2      # K % 8
+    assert g(vp(4096), vp(1 << 22), vp(1 << 24), 16, 12, 16, None) == 2      # N % 8
+    assert g(vp(4100), vp(1 << 22), vp(1 << 24), 16, 16, 16, None) == 2      # misaligned A
+    assert g(vp(4096), vp(1 << 22), vp(4096 + 64), 16, 16, 16, None) == 1    # C overlaps A
+    assert g(None, vp(1 << 22), vp(1 << 24), 16, 16, 16, None) == 1
+    assert g(None, None, None, 0, 16, 16, None) == 0                          # empty: nothing to do
     # the failure-path self-check takes limits of 1 ns .. 1 s only
     cuda_lib.hstu_attn_selfcheck_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     assert cuda_lib.hstu_attn_selfcheck_wait_timeout(0, None) == 1
