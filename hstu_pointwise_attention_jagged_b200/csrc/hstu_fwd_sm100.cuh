@@ -6,10 +6,11 @@
 //
 //   warp 8      producer: fetches the next item, TMA-loads Q (both halves) and the item's key
 //               tiles K_t, V_t into a ring of shared-memory stages (128B/64B swizzle).
-//   warp 9      MMA issuer (one thread): S_h = Q_h K_t^T into TMEM (SS form), then, once the
-//               SiLU warps have written P_h, O_h += P_h V_t with P_h read from TMEM (TS form).
-//               Issue order per key tile: PV_0(prev) S_0(t) PV_1(prev) S_1(t), so the tensor
-//               core always has the other half's work while one half's SiLU runs.
+//   warp 9      MMA issuer: the warp runs converged and lane 0 issues every tcgen05 instruction.
+//               S_h = Q_h K_t^T into TMEM (SS form), then, once the SiLU warps have written P_h,
+//               O_h += P_h V_t with P_h read from TMEM (TS form).  Issue order per key tile:
+//               PV_0(prev) S_0(t) PV_1(prev) S_1(t), so the tensor core has the other half's work
+//               while one half's SiLU runs.
 //   warps 0-3   SiLU warpgroup of half 0, warps 4-7 of half 1: TMEM -> registers, p =
 //               mask ? silu(alpha*s) : 0 with silu(x) = h + h*tanh(h), h = x/2 (one MUFU op per
 //               score), packed to bf16 and written back over S in TMEM; after the item's last
@@ -17,6 +18,10 @@
 //
 // TMEM (512 columns x 128 lanes of fp32): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
 // O_1 [256+D, 256+2D).  P_h (bf16 pairs) overwrites the first 64 columns of S_h.
+//
+// hstu_fwd_kernel<D, true> is the relative-attention-bias variant: each visible pair's p also gets
+// a per-head table entry for its query-key distance (the table is read through the read-only
+// cache); everything else is the same kernel.
 //
 // Every mbarrier wait is bounded by %globaltimer; on expiry the kernel records kErrTimeout,
 // raises a CTA-wide abort flag, lets every role leave its loop, drains the copies and MMAs it
@@ -161,10 +166,17 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t tad
     float p0 = fmaf(h0, ptx::tanh_approx(h0), h0);
     float p1 = fmaf(h1, ptx::tanh_approx(h1), h1);
     if constexpr (kRab) {
-      // Distances of masked pairs can be negative: clamp so the read stays inside the table.
-      const int d0 = rel0 - (kChunk * 32 + 2 * e);
-      p0 += __ldg(rab_row + min(max(d0, 0), rab_max));
-      p1 += __ldg(rab_row + min(max(d0 - 1, 0), rab_max));
+      // The chunk's distances run down from hi = rel0 - 32*chunk by one per column.  Inside the
+      // table the reads are fixed offsets from one base; otherwise (masked pairs have negative
+      // distances, far pairs exceed the table) each index is clamped into it.
+      const int hi = rel0 - kChunk * 32;
+      if (hi >= 31 && hi <= rab_max) {
+        p0 += __ldg(rab_row + hi - 2 * e);
+        p1 += __ldg(rab_row + hi - 2 * e - 1);
+      } else {
+        p0 += __ldg(rab_row + min(max(hi - 2 * e, 0), rab_max));
+        p1 += __ldg(rab_row + min(max(hi - 2 * e - 1, 0), rab_max));
+      }
     }
     if (!full) {
       const int c0 = kChunk * 32 + 2 * e;
