@@ -14,8 +14,9 @@
 //                waits and commits) into one of two TMEM accumulators of 256 columns;
 //   warps 2..5   epilogue: TMEM -> registers -> bf16 -> row- and column-predicated 16-byte stores,
 //                overlapping the next tile's main loop on the other accumulator.
-// Output tiles are visited in M-fastest order, so CTAs working at the same time share W tiles in
-// L2.  Every wait is bounded; a timeout sets the error word and the kernel drains and returns.
+// Output tiles are visited in N-fastest order: CTAs working at the same time share one A tile (the
+// large operand: token rows), while W, a few MB for a layer's projection, stays in L2 throughout.
+// Every wait is bounded; a timeout sets the error word and the kernel drains and returns.
 #pragma once
 
 #include "hstu_fwd_sm100.cuh"
@@ -101,8 +102,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % p.tiles_m) * kGemmBM;
-        const int n0 = (tile / p.tiles_m) * kGemmBN;
+        const int m0 = (tile / p.tiles_n) * kGemmBM;
+        const int n0 = (tile % p.tiles_n) * kGemmBN;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!wait_bounded(bar(ctl->empty[stage]), phase ^ 1u, abort_flag, p.err)) {
             ok = false;
@@ -174,8 +175,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok) break;
       acc_full_par[acc] ^= 1u;
       ptx::tc_fence_after();
-      const int m = (tile % p.tiles_m) * kGemmBM + row;
-      const int n0 = (tile / p.tiles_m) * kGemmBN;
+      const int m = (tile / p.tiles_n) * kGemmBM + row;
+      const int n0 = (tile % p.tiles_n) * kGemmBN;
       __nv_bfloat16* dst = p.c + (size_t)(m < p.M ? m : 0) * p.N + n0;
 #pragma unroll 1
       for (int c = 0; c < kGemmBN / 32; ++c) {
