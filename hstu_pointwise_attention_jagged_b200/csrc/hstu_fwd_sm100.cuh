@@ -489,19 +489,36 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const int self = i_pos - j0;
         const int rel0 = i_pos - j0;
         // 32-column chunks: the load of chunk c+1 is in flight while chunk c is computed.
-        uint32_t ra[32], rb[32];
-        ptx::tmem_ld32(taddr_s + 0, ra);
-        ptx::tmem_ld_wait(ra);
-        ptx::tmem_ld32(taddr_s + 32, rb);
-        silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-        ptx::tmem_ld_wait(rb);
-        ptx::tmem_ld32(taddr_s + 64, ra);
-        silu_chunk<1, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-        ptx::tmem_ld_wait(ra);
-        ptx::tmem_ld32(taddr_s + 96, rb);
-        silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-        ptx::tmem_ld_wait(rb);
-        silu_chunk<3, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+        if constexpr (kRab) {
+          // The bias reads need registers the next chunk's load would hold: one chunk at a time.
+          uint32_t ra[32];
+          ptx::tmem_ld32(taddr_s + 0, ra);
+          ptx::tmem_ld_wait(ra);
+          silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          ptx::tmem_ld32(taddr_s + 32, ra);
+          ptx::tmem_ld_wait(ra);
+          silu_chunk<1, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          ptx::tmem_ld32(taddr_s + 64, ra);
+          ptx::tmem_ld_wait(ra);
+          silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          ptx::tmem_ld32(taddr_s + 96, ra);
+          ptx::tmem_ld_wait(ra);
+          silu_chunk<3, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+        } else {
+          uint32_t ra[32], rb[32];
+          ptx::tmem_ld32(taddr_s + 0, ra);
+          ptx::tmem_ld_wait(ra);
+          ptx::tmem_ld32(taddr_s + 32, rb);
+          silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          ptx::tmem_ld_wait(rb);
+          ptx::tmem_ld32(taddr_s + 64, ra);
+          silu_chunk<1, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          ptx::tmem_ld_wait(ra);
+          ptx::tmem_ld32(taddr_s + 96, rb);
+          silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          ptx::tmem_ld_wait(rb);
+          silu_chunk<3, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+        }
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();
