@@ -35,7 +35,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "jagged SiLU-attention TFLOP/s & target tokens/s, % of B200 BF16 TC peak"
-WORKLOAD = "dlrmv3"
+WORKLOAD = "dlrmv3"  # the benchmark batch; --workload times one of the parity workloads instead
+WORKLOAD_SEEDS = {"dlrmv3": 1, "jagged": 2, "long_history": 3, "streaming": 4}
 FALLBACK_PEAK_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
 RAB_LEN = 4096  # relative-bias table entries per head for --variant rab
@@ -181,9 +182,13 @@ def profiled_traffic():
 
 
 def workload_config(w, n_gpus):
+    if w.name == WORKLOAD:
+        name = "%s: %d users x (%d history + %d candidates), H=%d, d=%d, alpha=1/sqrt(%d), N=%d" % (
+            w.name, w.B, int(w.uih_len[0]), int(w.num_targets[0]), w.H, w.d, w.d, int(w.N))
+    else:
+        name = "%s: %s" % (w.name, w.meta.get("description", ""))
     return {
-        "workload": "%s: %d users x (%d history + %d candidates), H=%d, d=%d, alpha=1/sqrt(%d), N=%d" % (
-            w.name, w.B, int(w.uih_len[0]), int(w.num_targets[0]), w.H, w.d, w.d, int(w.N)),
+        "workload": name,
         "users_per_gpu": w.B,
         "global_batch": w.B * n_gpus,
         "seq_len": int(w.seq_len.max()),
@@ -222,20 +227,25 @@ def run_ours(args, ranks):
     dev = torch.device("cuda", ranks.local_rank)
     torch.cuda.set_device(dev)
     binding.load_library()
-    w = workloads.make(WORKLOAD, seed=rank_seed(1, ranks.rank))
-    flops = metrics.algorithmic_flops(w.seq_offsets, w.num_targets, w.H, w.d)
+    w = workloads.make(args.workload, seed=rank_seed(WORKLOAD_SEEDS[args.workload], ranks.rank))
+    cached = bool(w.cached_len.any())
+    flops = metrics.algorithmic_flops(w.seq_offsets, w.num_targets, w.H, w.d, w.cached_len if cached else None)
     targets = int(w.num_targets.sum())
 
     def to_bf16(x):
         return torch.from_numpy(workloads.bf16_bits(x).view(np.int16)).view(torch.bfloat16)
 
-    q_h, k_h, v_h = (to_bf16(x).pin_memory() for x in (w.q, w.k, w.v))
+    # With a cached prefix (the streaming workload) the queries are the new tokens only.
+    q_rows = w.q[w.new_rows()] if cached else w.q
+    q_h, k_h, v_h = (to_bf16(x).pin_memory() for x in (q_rows, w.k, w.v))
     off_h = torch.from_numpy(w.seq_offsets.astype(np.int32)).pin_memory()
     nt_h = torch.from_numpy(w.num_targets.astype(np.int32)).pin_memory()
     q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
     off, nt = off_h.to(dev), nt_h.to(dev)
+    cl = torch.from_numpy(w.cached_len.astype(np.int32)).to(dev) if cached else None
+    total_q = int(q_h.shape[0])
     out = torch.empty_like(q)
-    plan = torch.empty((binding.hstu_attn_plan_bytes(w.B, w.H, w.total),), dtype=torch.uint8, device=dev)
+    plan = torch.empty((binding.hstu_attn_plan_bytes(w.B, w.H, total_q),), dtype=torch.uint8, device=dev)
     flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     msl = w.max_seq_len
@@ -248,13 +258,13 @@ def run_ours(args, ranks):
 
     def attn():
         if rab is None:
-            binding.hstu_attn_fwd_planned(q, k, v, off, nt, None, w.alpha, w.N, plan, out=out, stream=stream)
+            binding.hstu_attn_fwd_planned(q, k, v, off, nt, cl, w.alpha, w.N, plan, out=out, stream=stream)
         else:
-            binding.hstu_attn_fwd_rab(q, k, v, off, nt, rab, w.alpha, w.N, msl, out=out, stream=stream)
+            binding.hstu_attn_fwd_rab(q, k, v, off, nt, rab, w.alpha, w.N, msl, cached_len=cl, out=out, stream=stream)
 
     def step():
         if rab is None:
-            binding.hstu_attn_plan(off, nt, None, w.H, w.total, w.total, msl, plan=plan, stream=stream)
+            binding.hstu_attn_plan(off, nt, cl, w.H, w.total, total_q, msl, plan=plan, stream=stream)
         attn()
 
     for _ in range(args.warmup):
@@ -323,10 +333,13 @@ def run_ours(args, ranks):
             vd.copy_(v_h, non_blocking=True)
             od.copy_(off_h, non_blocking=True)
             nd.copy_(nt_h, non_blocking=True)
-            if rab is None:
-                binding.hstu_attn_fwd(qd, kd, vd, od, nd, w.alpha, w.N, msl, out=outd, stream=streams[j])
+            if rab is not None:
+                binding.hstu_attn_fwd_rab(qd, kd, vd, od, nd, rab, w.alpha, w.N, msl, cached_len=cl, out=outd,
+                                          stream=streams[j])
+            elif cached:
+                binding.hstu_attn_fwd_cached(qd, kd, vd, od, nd, cl, w.alpha, w.N, msl, out=outd, stream=streams[j])
             else:
-                binding.hstu_attn_fwd_rab(qd, kd, vd, od, nd, rab, w.alpha, w.N, msl, out=outd, stream=streams[j])
+                binding.hstu_attn_fwd(qd, kd, vd, od, nd, w.alpha, w.N, msl, out=outd, stream=streams[j])
             outs_h[j].copy_(outd, non_blocking=True)
 
     for i in range(4):
@@ -370,16 +383,18 @@ def run_ours(args, ranks):
         "algorithmic_gflop_per_step": round(job_flops / 1e9, 3),
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                "api": "hstu_attn_fwd (plan + attention) with pinned host buffers",
+                "api": "%s (plan + attention) with pinned host buffers" % (
+                    "hstu_attn_fwd_rab" if rab is not None else "hstu_attn_fwd_cached" if cached else "hstu_attn_fwd"),
                 "pipelining": "2 streams, double-buffered device tensors: uploads, kernels and downloads of "
                               "neighbouring steps overlap; %d steps" % E},
         "gpu_launches": (3 * K if rab is None else 4 * K) + 2 * E,
         "roofline": {"bound": "tensor",
-                     "kernel": "hstu_fwd_kernel<128, 0>" if rab is None else "hstu_fwd_kernel<128, rab> (+ plan kernel)",
+                     "kernel": ("hstu_fwd_kernel<%d, 0>" % w.d) if rab is None else (
+                         "hstu_fwd_kernel<%d, rab> (+ plan kernel)" % w.d),
                      "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": args.traffic if args.traffic is not None else (
-                         profiled_traffic() if rab is None else None),
+                         profiled_traffic() if rab is None and args.workload == WORKLOAD else None),
                      "peak_source": peak_src,
                      "attn_ms_per_launch": round(attn_avg_ms, 5),
                      "timing": ("attention kernel alone, %d launches on one plan, L2 flushed before each" % K
@@ -392,11 +407,15 @@ def run_ours(args, ranks):
         import oracle
         cores = oracle.num_threads()
         t0 = time.perf_counter()
-        if rab is None:
-            _, macs = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N, return_macs=True)
-        else:
-            oracle.fwd_rab(w.q, w.k, w.v, w.seq_offsets, w.num_targets, rab.cpu().numpy(), w.alpha, w.N)
+        if rab is not None:
+            oracle.fwd_rab(q_rows, w.k, w.v, w.seq_offsets, w.num_targets, rab.cpu().numpy(), w.alpha, w.N,
+                           cached_len=w.cached_len if cached else None)
             macs = flops // 2
+        elif cached:
+            _, macs = oracle.fwd_cached(q_rows, w.k, w.v, w.seq_offsets, w.num_targets, w.cached_len, w.alpha, w.N,
+                                        return_macs=True)
+        else:
+            _, macs = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N, return_macs=True)
         dt = time.perf_counter() - t0
         line["cpu_baseline"] = {"value": 2 * macs / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                 "sample": "one full step: every row and head of the same batch (fp64 C oracle, "
@@ -575,6 +594,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ref-rows", type=int, default=0, help="rows per step of the reference arm (0: sized from K)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_SEEDS), default=WORKLOAD,
+                    help="batch to time (default: the DLRMv3-shaped benchmark batch)")
     ap.add_argument("--variant", choices=["plain", "rab", "proj"], default="plain",
                     help="rab: the relative-attention-bias variant (a %d-entry table per head); proj: the layer's "
                          "projection GEMMs" % RAB_LEN)
