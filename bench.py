@@ -200,11 +200,13 @@ def workload_config(w, n_gpus):
 
 
 def oracle_sample_rows(w, n_rows, seed):
-    """A stratified sample of query rows (history and candidates in proportion) of the workload."""
+    """A sample of query rows of the workload: users uniformly among those with query rows, rows
+    uniformly within each (with a cached prefix, among the new tokens only)."""
     rng = np.random.default_rng(seed)
-    users = rng.integers(0, w.B, size=n_rows)
-    L = w.seq_len[users]
-    local = (rng.random(n_rows) * L).astype(np.int64)
+    nq = w.seq_len - w.cached_len
+    live = np.flatnonzero(nq > 0)
+    users = live[rng.integers(0, len(live), size=n_rows)]
+    local = (rng.random(n_rows) * nq[users]).astype(np.int64)
     return users.astype(np.int32), local.astype(np.int32)
 
 
@@ -212,9 +214,11 @@ def time_oracle(w, n_rows, seed):
     """Runs the oracle on a row sample; returns (seconds, algorithmic flops of the sample)."""
     import oracle
     users, local = oracle_sample_rows(w, n_rows, seed)
+    cached = bool(w.cached_len.any())
+    q = w.q[w.new_rows()] if cached else w.q
     t0 = time.perf_counter()
-    _, macs = oracle.rows(w.q, w.k, w.v, w.seq_offsets, w.num_targets, None, w.alpha, w.N, users, local,
-                          return_macs=True)
+    _, macs = oracle.rows(q, w.k, w.v, w.seq_offsets, w.num_targets, w.cached_len if cached else None, w.alpha,
+                          w.N, users, local, return_macs=True)
     dt = time.perf_counter() - t0
     return dt, 2 * macs
 
@@ -552,7 +556,7 @@ def run_reference(args, world):
     warm-up plus K steps stay near a minute of CPU work."""
     import oracle
     from hstu_pointwise_attention_jagged_b200 import workloads
-    w = workloads.make(WORKLOAD, seed=rank_seed(1, 0))
+    w = workloads.make(args.workload, seed=rank_seed(WORKLOAD_SEEDS[args.workload], 0))
     cores = oracle.num_threads()
     rows = args.ref_rows or int(min(8000, max(16, 240000 // (args.steps + args.warmup))))
     for i in range(args.warmup):
