@@ -12,7 +12,8 @@
 //   warp 1       MMA issuer: per 64-deep k block four tcgen05.mma 128×256×16 (each instruction
 //                carries 128 clocks of tensor work, so the issuing thread has slack for its
 //                waits and commits) into one of two TMEM accumulators of 256 columns;
-//   warps 2..5   epilogue: TMEM -> registers -> bf16 -> row- and column-predicated 16-byte stores,
+//   warps 2..5   epilogue: TMEM -> registers -> bf16 -> row- and column-predicated 32-byte stores
+//                (16-byte ones when N is not a multiple of 16 or C is not 32-byte aligned),
 //                overlapping the next tile's main loop on the other accumulator.
 // Output tiles are visited in N-fastest order: CTAs working at the same time share one A tile (the
 // large operand: token rows), while W, a few MB for a layer's projection, stays in L2 throughout.
@@ -51,6 +52,13 @@ struct GemmParams {
   int32_t tiles_m, tiles_n;
   unsigned* err;
 };
+
+// 32 bytes to global memory in one instruction (st.global.v8.b32); the address is 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint4& a, const uint4& b) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x), "r"(a.y),
+               "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
@@ -169,6 +177,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     uint32_t acc_full_par[2] = {0u, 0u};
     int acc = 0;
+    // 32-byte stores fill whole sectors; they need N % 16 == 0 and a 32-byte aligned C.
+    const bool wide_stores = (p.N % 16 == 0) && ((reinterpret_cast<uintptr_t>(p.c) & 31u) == 0);
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
       ok = __all_sync(0xffffffffu, wait_bounded(bar(ctl->acc_full[acc]), acc_full_par[acc], abort_flag, p.err));
@@ -184,17 +194,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ptx::tmem_ld32(tmem + lane_off + acc * kGemmBN + c * 32, r);
         ptx::tmem_ld_wait(r);
         if (m < p.M) {
+          uint4 v[4];
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
-            const int n = n0 + c * 32 + q4 * 8;
-            if (n < p.N) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
-              v.y = pack_bf16x2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
-              v.z = pack_bf16x2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
-              v.w = pack_bf16x2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
-              *reinterpret_cast<uint4*>(dst + c * 32 + q4 * 8) = v;
-            }
+            v[q4].x = pack_bf16x2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
+            v[q4].y = pack_bf16x2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
+            v[q4].z = pack_bf16x2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
+            v[q4].w = pack_bf16x2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
+          }
+          if (wide_stores) {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2)
+              if (n0 + c * 32 + h2 * 16 < p.N) st_global_v8(dst + c * 32 + h2 * 16, v[2 * h2], v[2 * h2 + 1]);
+          } else {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              if (n0 + c * 32 + q4 * 8 < p.N) *reinterpret_cast<uint4*>(dst + c * 32 + q4 * 8) = v[q4];
           }
         }
       }
