@@ -13,7 +13,9 @@ depends on a candidate, and target-aware attention weighs history against each c
     out[i,h,:] = (1/N) * sum_{j in A(i)} silu(alpha * q[i,h,:].k[j,h,:]) * v[j,h,:]
     A(i) = {j <= i} for a history token (i < U); {j < U} + {i} for a candidate (i >= U)
 
-The C source (``hstu_oracle.c``) holds the arithmetic; this module only marshals numpy arrays.
+The backward pass (``bwd``, ``bwd_rows``) is derived from that definition by the chain rule; the
+pages print none.  The C source (``hstu_oracle.c``) holds the arithmetic; this module only marshals
+numpy arrays.
 """
 import ctypes
 import os
@@ -40,8 +42,13 @@ class Oracle:
                                          i64, f64, f64, i32p, i32p, i64, f64p, i64p]
         lib.hstu_oracle_rows_rab.argtypes = [f32p, f32p, f32p, i32p, i32p, i32p, f32p, i32, i32, i32,
                                              i32, i64, i64, f64, f64, i32p, i32p, i64, f64p]
+        lib.hstu_oracle_bwd.argtypes = [f32p, f32p, f32p, f32p, i32p, i32p, i32, i32, i32, i64, f64, f64,
+                                        f64p, f64p, f64p]
+        lib.hstu_oracle_bwd_rows.argtypes = [f32p, f32p, f32p, f32p, i32p, i32p, i32, i32, i32, i64, f64, f64,
+                                             i32p, i32p, i64, f64p, f64p, f64p]
         for fn in (lib.hstu_oracle_fwd, lib.hstu_oracle_fwd_cached, lib.hstu_oracle_rows,
-                   lib.hstu_oracle_rows_rab, lib.hstu_oracle_num_threads):
+                   lib.hstu_oracle_rows_rab, lib.hstu_oracle_num_threads, lib.hstu_oracle_bwd,
+                   lib.hstu_oracle_bwd_rows):
             fn.restype = ctypes.c_int
         self.lib = lib
 
@@ -140,6 +147,43 @@ class Oracle:
         return self.rows_rab(q, k, v, seq_offsets, num_targets, cached_len, rab, alpha, N, users, local)
 
 
+    def bwd(self, q, k, v, dout, seq_offsets, num_targets, alpha, N):
+        """Backward pass of the full forward: returns (dq, dk, dv), float64 [total, H, d] each, for
+        the loss gradient dout [total, H, d] with respect to out."""
+        q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
+        off = _i32(seq_offsets)
+        nt = None if num_targets is None else _i32(num_targets)
+        total, H, d = q.shape
+        dq, dk, dv = (np.zeros((total, H, d), dtype=np.float64) for _ in range(3))
+        rc = self.lib.hstu_oracle_bwd(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float),
+                                      _ptr(dout, ctypes.c_float), _ptr(off, ctypes.c_int32),
+                                      _ptr(nt, ctypes.c_int32), len(off) - 1, H, d, total, float(alpha),
+                                      float(N), _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
+                                      _ptr(dv, ctypes.c_double))
+        if rc != 0:
+            raise ValueError("oracle: inconsistent seq_offsets / num_targets")
+        return dq, dk, dv
+
+    def bwd_rows(self, q, k, v, dout, seq_offsets, num_targets, alpha, N, row_user, row_local):
+        """Selected rows of the backward pass: for each (user, position) pair, dq of that query row
+        and dk, dv of that key row ([n, H, d] float64 each), equal to the full pass's rows."""
+        q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
+        off = _i32(seq_offsets)
+        nt = None if num_targets is None else _i32(num_targets)
+        ru, rl = _i32(row_user), _i32(row_local)
+        total, H, d = q.shape
+        dq, dk, dv = (np.zeros((len(ru), H, d), dtype=np.float64) for _ in range(3))
+        rc = self.lib.hstu_oracle_bwd_rows(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                           _ptr(v, ctypes.c_float), _ptr(dout, ctypes.c_float),
+                                           _ptr(off, ctypes.c_int32), _ptr(nt, ctypes.c_int32), len(off) - 1, H, d,
+                                           total, float(alpha), float(N), _ptr(ru, ctypes.c_int32),
+                                           _ptr(rl, ctypes.c_int32), len(ru), _ptr(dq, ctypes.c_double),
+                                           _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double))
+        if rc != 0:
+            raise ValueError("oracle: inconsistent offsets or row selection")
+        return dq, dk, dv
+
+
 def _f32(a):
     return np.ascontiguousarray(a, dtype=np.float32)
 
@@ -187,6 +231,14 @@ def rows_rab(*args, **kwargs):
 
 def fwd_rab(*args, **kwargs):
     return default().fwd_rab(*args, **kwargs)
+
+
+def bwd(*args, **kwargs):
+    return default().bwd(*args, **kwargs)
+
+
+def bwd_rows(*args, **kwargs):
+    return default().bwd_rows(*args, **kwargs)
 
 
 def linear(a, w):

@@ -298,3 +298,172 @@ int hstu_oracle_rows_rab(const float* q, const float* k, const float* v,
   free(qstart);
   return 0;
 }
+
+/*
+ * ---------------------------------------------------------------------------------------------
+ * Backward pass.  The pages print no backward pass; the training story they tell (the scaling
+ * section of the infolabhq.com multi-stage page) needs one.  It is derived here from the
+ * forward definition above by the chain rule, for a scalar loss whose gradient with respect to
+ * out is dout:
+ *
+ *   for every user, head, query position i and visible key j in A(i):
+ *     s   = sum_c q[i,c] k[j,c],   x = alpha * s
+ *     p   = silu(x)                        dv[j,:] += p * dout[i,:] / N
+ *     g   = sum_c dout[i,c] v[j,c] / N     (gradient of the loss with respect to p)
+ *     ds  = g * silu'(x) * alpha           (gradient with respect to s)
+ *                                          dq[i,:] += ds * k[j,:]
+ *                                          dk[j,:] += ds * q[i,:]
+ *   silu'(x) = sigma(x) * (1 + x * (1 - sigma(x))),  sigma(x) = 1 / (1 + exp(-x))
+ *
+ * Masked pairs contribute nothing to any gradient.  Order: queries i ascending, and within a
+ * query its keys j ascending, for every sum, so dq[i] adds keys in ascending order and dk[j],
+ * dv[j] add queries in ascending order.
+ * ---------------------------------------------------------------------------------------------
+ */
+
+/* Derivative of silu(x) = x * sigma(x): sigma(x) + x * sigma(x) * (1 - sigma(x)). */
+static double dsilu(double x) {
+  double sg = 1.0 / (1.0 + exp(-x));
+  return sg * (1.0 + x * (1.0 - sg));
+}
+
+/*
+ * Gradients of one user and head.  qs, ks, vs, dos: first row of the user's segment (row
+ * stride `stride` floats, already offset to the head); dqs, dks, dvs: the same for the
+ * doubles written (zeroed here first).  L: segment length; U: history length.
+ */
+static void bwd_user_head(const float* qs, const float* ks, const float* vs, const float* dos,
+                          int64_t stride, int32_t d, int32_t L, int32_t U, double alpha, double N,
+                          double* dqs, double* dks, double* dvs) {
+  for (int32_t t = 0; t < L; ++t)
+    for (int32_t c = 0; c < d; ++c) {
+      dqs[(int64_t)t * stride + c] = 0.0;
+      dks[(int64_t)t * stride + c] = 0.0;
+      dvs[(int64_t)t * stride + c] = 0.0;
+    }
+  for (int32_t i = 0; i < L; ++i) {
+    const float* qi = qs + (int64_t)i * stride;
+    const float* doi = dos + (int64_t)i * stride;
+    double* dqi = dqs + (int64_t)i * stride;
+    for (int32_t j = 0; j < L; ++j) {
+      if (!visible(i, j, U)) continue;
+      const float* kj = ks + (int64_t)j * stride;
+      const float* vj = vs + (int64_t)j * stride;
+      double* dkj = dks + (int64_t)j * stride;
+      double* dvj = dvs + (int64_t)j * stride;
+      double s = 0.0, g = 0.0;
+      for (int32_t c = 0; c < d; ++c) s += (double)qi[c] * (double)kj[c];
+      for (int32_t c = 0; c < d; ++c) g += (double)doi[c] * (double)vj[c];
+      g /= N;
+      double x = alpha * s;
+      double p = silu(x);
+      double ds = g * dsilu(x) * alpha;
+      for (int32_t c = 0; c < d; ++c) {
+        dvj[c] += p * (double)doi[c] / N;
+        dqi[c] += ds * (double)kj[c];
+        dkj[c] += ds * (double)qi[c];
+      }
+    }
+  }
+}
+
+/*
+ * Full backward pass: dq, dk, dv [total, H, d] doubles from q, k, v, dout [total, H, d].
+ * Returns 0, or -1 on inconsistent offsets.
+ */
+int hstu_oracle_bwd(const float* q, const float* k, const float* v, const float* dout,
+                    const int32_t* seq_offsets, const int32_t* num_targets, int32_t B, int32_t H,
+                    int32_t d, int64_t total, double alpha, double N, double* dq, double* dk,
+                    double* dv) {
+  if (B < 0 || H <= 0 || d <= 0 || !(N != 0.0)) return -1;
+  if (seq_offsets[0] != 0 || seq_offsets[B] != total) return -1;
+  for (int32_t b = 0; b < B; ++b)
+    if (user_ok(seq_offsets, num_targets, NULL, b, total)) return -1;
+  const int64_t stride = (int64_t)H * d;
+  int64_t units = (int64_t)B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t u = 0; u < units; ++u) {
+    int32_t b = (int32_t)(u / H);
+    int32_t h = (int32_t)(u % H);
+    int32_t L = seq_offsets[b + 1] - seq_offsets[b];
+    int32_t T = num_targets ? num_targets[b] : 0;
+    int64_t o = (int64_t)seq_offsets[b] * stride + (int64_t)h * d;
+    bwd_user_head(q + o, k + o, v + o, dout + o, stride, d, L, L - T, alpha, N, dq + o, dk + o,
+                  dv + o);
+  }
+  return 0;
+}
+
+/*
+ * Selected rows of the backward pass, for checks at sizes where the full pass is too slow.
+ * For n in [0, nrows): user row_user[n], position row_local[n] of that user's segment; writes
+ * dq of that query row and dk, dv of that key row ([nrows, H, d] doubles each), each summed in
+ * the same order as hstu_oracle_bwd, so the rows equal the full pass's rows exactly.
+ * Returns 0, or -1 on inconsistent offsets or rows.
+ */
+int hstu_oracle_bwd_rows(const float* q, const float* k, const float* v, const float* dout,
+                         const int32_t* seq_offsets, const int32_t* num_targets, int32_t B,
+                         int32_t H, int32_t d, int64_t total, double alpha, double N,
+                         const int32_t* row_user, const int32_t* row_local, int64_t nrows,
+                         double* dq, double* dk, double* dv) {
+  if (B < 0 || H <= 0 || d <= 0 || !(N != 0.0)) return -1;
+  if (seq_offsets[0] != 0 || seq_offsets[B] != total) return -1;
+  for (int32_t b = 0; b < B; ++b)
+    if (user_ok(seq_offsets, num_targets, NULL, b, total)) return -1;
+  for (int64_t n = 0; n < nrows; ++n) {
+    int32_t b = row_user[n];
+    if (b < 0 || b >= B) return -1;
+    if (row_local[n] < 0 || row_local[n] >= seq_offsets[b + 1] - seq_offsets[b]) return -1;
+  }
+  const int64_t stride = (int64_t)H * d;
+  int64_t units = nrows * H;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t u = 0; u < units; ++u) {
+    int64_t n = u / H;
+    int32_t h = (int32_t)(u % H);
+    int32_t b = row_user[n];
+    int32_t L = seq_offsets[b + 1] - seq_offsets[b];
+    int32_t U = L - (num_targets ? num_targets[b] : 0);
+    int32_t r = row_local[n];
+    int64_t o = (int64_t)seq_offsets[b] * stride + (int64_t)h * d;
+    const float *qs = q + o, *ks = k + o, *vs = v + o, *dos = dout + o;
+    double* dqn = dq + n * stride + (int64_t)h * d;
+    double* dkn = dk + n * stride + (int64_t)h * d;
+    double* dvn = dv + n * stride + (int64_t)h * d;
+    for (int32_t c = 0; c < d; ++c) dqn[c] = dkn[c] = dvn[c] = 0.0;
+    /* dq of query row r: its visible keys, ascending */
+    const float* qi = qs + (int64_t)r * stride;
+    const float* doi = dos + (int64_t)r * stride;
+    for (int32_t j = 0; j < L; ++j) {
+      if (!visible(r, j, U)) continue;
+      const float* kj = ks + (int64_t)j * stride;
+      const float* vj = vs + (int64_t)j * stride;
+      double s = 0.0, g = 0.0;
+      for (int32_t c = 0; c < d; ++c) s += (double)qi[c] * (double)kj[c];
+      for (int32_t c = 0; c < d; ++c) g += (double)doi[c] * (double)vj[c];
+      g /= N;
+      double ds = g * dsilu(alpha * s) * alpha;
+      for (int32_t c = 0; c < d; ++c) dqn[c] += ds * (double)kj[c];
+    }
+    /* dk, dv of key row r: the queries that see it, ascending */
+    const float* kr = ks + (int64_t)r * stride;
+    const float* vr = vs + (int64_t)r * stride;
+    for (int32_t i = 0; i < L; ++i) {
+      if (!visible(i, r, U)) continue;
+      const float* qi2 = qs + (int64_t)i * stride;
+      const float* doi2 = dos + (int64_t)i * stride;
+      double s = 0.0, g = 0.0;
+      for (int32_t c = 0; c < d; ++c) s += (double)qi2[c] * (double)kr[c];
+      for (int32_t c = 0; c < d; ++c) g += (double)doi2[c] * (double)vr[c];
+      g /= N;
+      double x = alpha * s;
+      double p = silu(x);
+      double ds = g * dsilu(x) * alpha;
+      for (int32_t c = 0; c < d; ++c) {
+        dvn[c] += p * (double)doi2[c] / N;
+        dkn[c] += ds * (double)qi2[c];
+      }
+    }
+  }
+  return 0;
+}
