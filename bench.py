@@ -6,9 +6,10 @@ One step = one forward pass of the attention (work plan + attention kernel) over
 the DLRMv3-shaped workload: 8 users x (2048 history + 2048 candidate tokens), H=4 heads of
 d=128, bf16 N(0,1)/sqrt(d) inputs, alpha=1/sqrt(128), N=4096 (synthetic: the DLRMv3 dataset is
 not available).  Inputs are resident in HBM; L2 is flushed (256 MiB write) before every timed
-step.  Multi-GPU: one process per GPU, each with its own batch (users are independent, so the
-batch is sharded by user with no collective on the data path; weak scaling); the only
-collectives are the barrier and the max-over-ranks of the device time.
+step.  Multi-GPU: one process per GPU; the global batch is N replicas of the workload's users,
+split by hstu_attn_partition into contiguous runs of equal visible-pair cost, one per GPU (users
+are independent, so there is no collective on the data path; per-GPU work is fixed: weak
+scaling); the only collectives are the barrier and the max/sum over ranks of the timings.
 
 Prints one JSON line on rank 0.  `value` is whole-job algorithmic TFLOP/s (visible query/key
 pairs only, both matmuls); `e2e` is the same metric through the one-shot public entry point
@@ -38,6 +39,7 @@ METRIC = "jagged SiLU-attention TFLOP/s & target tokens/s, % of B200 BF16 TC pea
 WORKLOAD = "dlrmv3"  # the benchmark batch; --workload times one of the parity workloads instead
 WORKLOAD_SEEDS = {"dlrmv3": 1, "jagged": 2, "long_history": 3, "streaming": 4}
 FALLBACK_PEAK_TFLOPS = 1590.0
+DATASHEET_PEAK_TFLOPS = 2250.0  # NVIDIA's dense bf16 figure for one B200, for context beside the measured peak
 L2_FLUSH_BYTES = 256 << 20
 RAB_LEN = 4096  # relative-bias table entries per head for --variant rab
 
@@ -83,8 +85,32 @@ class Ranks:
 
 
 def rank_seed(base_seed: int, rank: int) -> int:
-    """Each rank draws its own batch of the same shape."""
+    """Seed of the r-th replica's lengths and of rank r's values."""
     return base_seed + 1000 * rank
+
+
+def rank_workload(name, world, rank):
+    """This rank's share of one global batch.  With one GPU it is the named workload itself.  With
+    N GPUs the global batch is N replicas of the workload's users (replica r's lengths drawn with
+    rank_seed(seed, r)); hstu_attn_partition splits it into contiguous runs of users of nearly equal
+    visible-pair cost, and this rank draws Q/K/V for its run.  Returns (workload, users in the
+    global batch)."""
+    from hstu_pointwise_attention_jagged_b200 import binding, workloads
+    base = WORKLOAD_SEEDS[name]
+    if world == 1:
+        w = workloads.make(name, seed=base)
+        return w, w.B
+    parts = [workloads.structure(name, seed=rank_seed(base, r)) for r in range(world)]
+    uih, nt, cl = (np.concatenate([p[i] for p in parts]) for i in range(3))
+    H, d, alpha, N = parts[0][3:]
+    off = workloads.offsets_from_lengths(uih + nt)
+    us = binding.hstu_attn_partition(off, nt, cl, world)
+    u0, u1 = int(us[rank]), int(us[rank + 1])
+    w = workloads.make_custom(name, uih[u0:u1], nt[u0:u1], H, d, alpha, N, seed=rank_seed(base, rank),
+                              cached_len=cl[u0:u1])
+    w.meta["description"] = workloads.CONFIGS[name][0]
+    w.meta["users"] = (u0, u1)
+    return w, len(uih)
 
 
 # ------------------------------------------------------------------------------------ clocks
@@ -181,7 +207,7 @@ def profiled_traffic():
     return int(rec["dram_bytes_per_launch"])
 
 
-def workload_config(w, n_gpus):
+def workload_config(w, n_gpus, global_users=None):
     if w.name == WORKLOAD:
         name = "%s: %d users x (%d history + %d candidates), H=%d, d=%d, alpha=1/sqrt(%d), N=%d" % (
             w.name, w.B, int(w.uih_len[0]), int(w.num_targets[0]), w.H, w.d, w.d, int(w.N))
@@ -190,11 +216,13 @@ def workload_config(w, n_gpus):
     return {
         "workload": name,
         "users_per_gpu": w.B,
-        "global_batch": w.B * n_gpus,
+        "global_batch": int(global_users if global_users is not None else w.B * n_gpus),
         "seq_len": int(w.seq_len.max()),
         "heads": w.H,
         "head_dim": w.d,
-        "parallelism": "dp%d (users sharded, no collective)" % n_gpus,
+        "parallelism": ("dp1" if n_gpus == 1 else
+                        "dp%d (one batch of %d x the workload's users split into contiguous runs of equal "
+                        "visible-pair cost by hstu_attn_partition; no collective)" % (n_gpus, n_gpus)),
         "l2": "flushed before every timed step (256 MiB write)",
     }
 
@@ -231,7 +259,7 @@ def run_ours(args, ranks):
     dev = torch.device("cuda", ranks.local_rank)
     torch.cuda.set_device(dev)
     binding.load_library()
-    w = workloads.make(args.workload, seed=rank_seed(WORKLOAD_SEEDS[args.workload], ranks.rank))
+    w, global_users = rank_workload(args.workload, ranks.world, ranks.rank)
     cached = bool(w.cached_len.any())
     flops = metrics.algorithmic_flops(w.seq_offsets, w.num_targets, w.H, w.d, w.cached_len if cached else None)
     targets = int(w.num_targets.sum())
@@ -280,10 +308,11 @@ def run_ours(args, ranks):
         raise RuntimeError("warm-up reported %s" % binding.hstu_attn_status_string(status))
 
     K = args.steps
-    # Two timed loops, K steps each, L2 flushed before every step.  The first times the whole
-    # hot path (plan + attention, no event between them, so the attention kernel's programmatic
-    # early launch overlaps the plan kernel as it does for a user); the second times the
-    # attention kernel alone on the same plan, for its roofline.
+    # One timed loop of K iterations, L2 flushed before every timed launch.  Each iteration times
+    # the whole hot path (plan + attention, no event between them, so the attention kernel's
+    # programmatic early launch overlaps the plan kernel as it does for a user), then the
+    # attention kernel alone on the same plan, for its roofline.  Interleaving the two makes both
+    # figures see the same clocks and the same state of the GPU.
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     eva = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
@@ -295,7 +324,6 @@ def run_ours(args, ranks):
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
-        for i in range(K):
             flush.zero_()
             eva[i][0].record(stream)
             attn()
@@ -380,7 +408,7 @@ def run_ours(args, ranks):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1)/sqrt(d) bf16; DLRMv3 dataset unavailable)",
-        "config": dict(workload_config(w, ranks.world), **({} if rab is None else {
+        "config": dict(workload_config(w, ranks.world, global_users), **({} if rab is None else {
             "variant": "relative attention bias: silu(alpha*s) + rab[h, min(i-j, %d)]" % (RAB_LEN - 1)})),
         "target_tokens_per_s": round(job_targets / (ms_per_step * 1e-3), 1),
         "pct_of_peak": round(100.0 * value / ranks.world / peak, 2),
@@ -397,6 +425,8 @@ def run_ours(args, ranks):
                          "hstu_fwd_kernel<%d, rab> (+ plan kernel)" % w.d),
                      "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "datasheet_peak": DATASHEET_PEAK_TFLOPS,
+                     "frac_of_datasheet": round(achieved / DATASHEET_PEAK_TFLOPS, 4),
                      "traffic": args.traffic if args.traffic is not None else (
                          profiled_traffic() if rab is None and args.workload == WORKLOAD else None),
                      "peak_source": peak_src,

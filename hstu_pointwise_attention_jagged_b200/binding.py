@@ -36,6 +36,8 @@ EXPORTS = (
     "hstu_attn_status_string",
     "hstu_attn_selfcheck_wait_timeout",
     "hstu_attn_gemm_bf16",
+    "hstu_attn_bwd",
+    "hstu_attn_partition",
 )
 
 
@@ -78,9 +80,12 @@ def load_library():
     lib.hstu_attn_status_string.argtypes = [ctypes.c_int]
     lib.hstu_attn_selfcheck_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.hstu_attn_gemm_bf16.argtypes = [vp, vp, vp, i32, i32, i32, vp]
+    lib.hstu_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp, vp]
+    lib.hstu_attn_partition.argtypes = [vp, vp, vp, i32, i32, vp]
     lib.hstu_attn_status_string.restype = ctypes.c_char_p
     for name in ("hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_fwd_rab", "hstu_attn_plan", "hstu_attn_fwd_planned",
-                 "hstu_attn_get_error", "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16"):
+                 "hstu_attn_get_error", "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16", "hstu_attn_bwd",
+                 "hstu_attn_partition"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -325,3 +330,58 @@ def hstu_attn_gemm_bf16(a, w, out=None, stream=None):
         st = lib.hstu_attn_gemm_bf16(_ptr(a), _ptr(w), _ptr(out), M, N, K, _stream_ptr(stream, a.device))
     _raise_if(st, "hstu_attn_gemm_bf16")
     return out
+
+
+def hstu_attn_bwd(q, k, v, dout, seq_offsets, num_targets, alpha, N, max_seq_len, dq=None, dk=None, dv=None,
+                  stream=None):
+    """Backward pass of hstu_attn_fwd; returns (dq, dk, dv), bf16 [total, H, d]. See include/hstu_attn.h."""
+    lib = load_library()
+    _check_tokens("q", q)
+    total, H, d = q.shape
+    for name, t in (("k", k), ("v", v), ("dout", dout)):
+        _check_tokens(name, t, H, d)
+        if t.shape[0] != total:
+            raise ValueError("q, k, v and dout must have the same number of rows")
+    B = seq_offsets.numel() - 1
+    _check_index("seq_offsets", seq_offsets, B + 1, q.device, optional=False)
+    _check_index("num_targets", num_targets, B, q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_tokens(name, t, H, d)
+    with torch.cuda.device(q.device):
+        st = lib.hstu_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(seq_offsets), _ptr(num_targets), B, H,
+                               d, total, int(max_seq_len), float(alpha), float(N), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _stream_ptr(stream, q.device))
+    _raise_if(st, "hstu_attn_bwd")
+    return dq, dk, dv
+
+
+def hstu_attn_partition(seq_offsets, num_targets, cached_len, parts):
+    """Contiguous user runs, one per GPU, minimising the largest visible-pair cost (host arrays in,
+    numpy int32 [parts+1] out: GPU p takes users [out[p], out[p+1])). See include/hstu_attn.h."""
+    import numpy as np
+    lib = load_library()
+    off = np.ascontiguousarray(seq_offsets, np.int32)
+    B = len(off) - 1
+    nt = None if num_targets is None else np.ascontiguousarray(num_targets, np.int32)
+    cl = None if cached_len is None else np.ascontiguousarray(cached_len, np.int32)
+    out = np.zeros(int(parts) + 1, np.int32)
+
+    def p(a):
+        return None if a is None else ctypes.c_void_p(a.ctypes.data)
+
+    st = lib.hstu_attn_partition(p(off), p(nt), p(cl), B, int(parts), p(out))
+    _raise_if(st, "hstu_attn_partition")
+    return out
+
+
+def shard_of(seq_offsets, user_start, part):
+    """Rows and rebased offsets of one GPU's run of users: (first user, last user + 1, first token
+    row, last token row + 1, seq_offsets of the run starting at 0)."""
+    import numpy as np
+    off = np.asarray(seq_offsets, np.int64)
+    u0, u1 = int(user_start[part]), int(user_start[part + 1])
+    r0, r1 = int(off[u0]), int(off[u1])
+    return u0, u1, r0, r1, (off[u0:u1 + 1] - r0).astype(np.int32)

@@ -1,0 +1,165 @@
+// bwd_schedule.cuh — device-side work lists of the backward pass.
+//
+// The backward pass of out = Mask(SiLU(alpha Q K^T)) V / N (DLRMv3 review, section "model
+// selection") runs as two persistent kernels over 128-row tiles of each user's segment:
+//   - the dK/dV kernel owns one key tile and streams the query tiles that see it:
+//       a history key tile (first key < U) is seen by every query tile from its own to the last
+//       (history queries at or after it, and every candidate); a candidate-only key tile is seen
+//       by its own query tile alone (a candidate sees itself among candidates);
+//   - the dQ kernel owns one query tile and streams its visible key tiles, the same runs as the
+//       forward pass.
+// Both lists are sorted by cost (streamed tiles per item), largest first, so the persistent
+// kernels run longest-processing-time-first.
+#pragma once
+
+#include <cstdint>
+
+#include "schedule.cuh"
+
+namespace hstu {
+
+// Query tiles that see key tile kt of a segment of L tokens with U history tokens, as a
+// TileRange ([0, e1) is always empty here).
+__host__ __device__ __forceinline__ TileRange query_tiles_of_key_tile(int kt, int L, int U) {
+  TileRange r{0, kt, kt + 1};
+  if (kt * kTileRows < U) r.e2 = cdiv(L, kTileRows);
+  return r;
+}
+
+// Key tiles visible to query tile qt (the forward pass's runs).
+__host__ __device__ __forceinline__ TileRange key_tiles_of_query_tile(int qt, int L, int U) {
+  const int p0 = qt * kTileRows;
+  const int p1 = (p0 + kTileRows < L) ? p0 + kTileRows : L;
+  return key_tiles(p0, p1, U);
+}
+
+struct BwdSchedArgs {
+  const int32_t* seq_offsets;  // [B+1]
+  const int32_t* num_targets;  // [B] or null
+  int32_t B, H, total, max_seq_len, nbins, max_items;
+  int32_t* header;      // [8] out: {dq counter, dq items, dq done, 0, kv counter, kv items, kv done, 0}
+  int32_t* tile_start;  // [B+1] out: index of each user's first 128-row tile among all tiles
+  int4* dq_items;       // [max_items] out: {b, query tile, h, cost}, non-increasing cost
+  int4* kv_items;       // [max_items] out: {b, key tile, h, cost}, non-increasing cost
+  unsigned* err;
+};
+
+// One CTA of kSchedThreads threads: validates every user (a bad user sets kErrBadOffsets and gets
+// no items), then writes both lists with a counting sort over cost bins.
+__global__ void __launch_bounds__(kSchedThreads) bwd_schedule_kernel(const BwdSchedArgs a) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ int hist[kMaxCostBins];
+  __shared__ long long scan_scratch[2][32];
+  __shared__ long long carry;
+  __shared__ int s_L[kCachedUsers], s_U[kCachedUsers], s_ts[kCachedUsers + 1];
+  const bool cached = a.B <= kCachedUsers;
+  const int tid = threadIdx.x;
+  const int nbins = a.nbins;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+
+  // Pass 1: validation and tile starts.
+  for (int base = 0; base < a.B; base += kSchedThreads) {
+    const int b = base + tid;
+    long long nt = 0, dummy = 0;
+    int L = 0, U = 0;
+    if (b < a.B) {
+      const int o0 = a.seq_offsets[b], o1 = a.seq_offsets[b + 1];
+      const long long L64 = (long long)o1 - o0;
+      const int T = a.num_targets ? a.num_targets[b] : 0;
+      bool ok = o0 >= 0 && L64 >= 0 && o1 <= a.total && L64 <= a.max_seq_len && T >= 0 && T <= L64;
+      if (b == 0 && o0 != 0) ok = false;
+      if (b == a.B - 1 && o1 != a.total) ok = false;
+      if (!ok) atomicOr(a.err, kErrBadOffsets);
+      L = ok ? (int)L64 : 0;
+      U = L - (ok ? T : 0);
+      nt = cdiv(L, kTileRows);
+    }
+    long long incl = nt, tot, tot2;
+    block_inclusive_scan2(incl, dummy, scan_scratch, tot, tot2);
+    const long long start = carry + incl - nt;
+    if (b < a.B) {
+      a.tile_start[b] = (int)start;
+      if (cached) {
+        s_L[b] = L;
+        s_U[b] = U;
+        s_ts[b] = (int)start;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) carry += tot;
+    __syncthreads();
+  }
+  const int ntiles = (int)carry;
+  if (tid == 0) {
+    a.tile_start[a.B] = ntiles;
+    if (cached) s_ts[a.B] = ntiles;
+  }
+  __syncthreads();
+
+  // Tile g: its user, its index within the user, and the user's L and U.  Users skipped in
+  // pass 1 own no tiles.
+  auto tile_of = [&](int g, int& b, int& t, int& L, int& U) {
+    b = owner_of(cached ? s_ts : a.tile_start, a.B, g);
+    t = g - (cached ? s_ts[b] : a.tile_start[b]);
+    if (cached) {
+      L = s_L[b];
+      U = s_U[b];
+    } else {
+      L = a.seq_offsets[b + 1] - a.seq_offsets[b];
+      U = L - (a.num_targets ? a.num_targets[b] : 0);
+    }
+  };
+
+  for (int list = 0; list < 2; ++list) {
+    int4* items = list == 0 ? a.dq_items : a.kv_items;
+    for (int i = tid; i < nbins; i += kSchedThreads) hist[i] = 0;
+    __syncthreads();
+    auto cost_of = [&](int t, int L, int U) {
+      return tile_count(list == 0 ? key_tiles_of_query_tile(t, L, U) : query_tiles_of_key_tile(t, L, U));
+    };
+    for (int g = tid; g < ntiles; g += kSchedThreads) {
+      int b, t, L, U;
+      tile_of(g, b, t, L, U);
+      const int c = cost_of(t, L, U);
+      atomicAdd(&hist[c < nbins ? c : nbins - 1], a.H);
+    }
+    __syncthreads();
+    const int per = cdiv(nbins, kSchedThreads);
+    long long part = 0;
+    for (int k = 0; k < per; ++k) {
+      const int bin = nbins - 1 - (tid * per + k);
+      if (bin >= 0) part += hist[bin];
+    }
+    __syncthreads();
+    long long tot;
+    const long long incl = block_inclusive_scan(part, scan_scratch[0], &tot);
+    long long run = incl - part;
+    for (int k = 0; k < per; ++k) {
+      const int bin = nbins - 1 - (tid * per + k);
+      if (bin >= 0) {
+        const int n = hist[bin];
+        hist[bin] = (int)run;
+        run += n;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      a.header[4 * list + 0] = 0;
+      a.header[4 * list + 1] = (int)(tot < a.max_items ? tot : a.max_items);
+      a.header[4 * list + 2] = 0;
+      a.header[4 * list + 3] = 0;
+    }
+    for (int g = tid; g < ntiles; g += kSchedThreads) {
+      int b, t, L, U;
+      tile_of(g, b, t, L, U);
+      const int c = cost_of(t, L, U);
+      const int pos = atomicAdd(&hist[c < nbins ? c : nbins - 1], a.H);
+      for (int h = 0; h < a.H; ++h)
+        if (pos + h < a.max_items) items[pos + h] = make_int4(b, t, h, c);
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace hstu

@@ -14,8 +14,10 @@
 #include <cstring>
 #include <functional>
 #include <mutex>
+#include <vector>
 
 #include "hstu_attn.h"
+#include "hstu_bwd_sm100.cuh"
 #include "hstu_fwd_sm100.cuh"
 #include "gemm_sm100.cuh"
 #include "schedule.cuh"
@@ -48,6 +50,12 @@ cudaError_t set_kernel_attrs() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(hstu_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              FwdCfg<D>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(hstu_bwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BwdCfg<D>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(hstu_bwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BwdCfg<D>::kSmemBytes);
   return e;
 }
 
@@ -311,6 +319,135 @@ hstu_status_t run(const void* q, const void* k, const void* v, const int32_t* se
   return s;
 }
 
+// Backward plan layout:
+//   int32 header[8] = {dq counter, dq items, dq done, 0, kv counter, kv items, kv done, 0}
+//   int32 tile_start[B+1], padded to 16 bytes
+//   int4  dq_items[cap], kv_items[cap], cap = H * (total / 128 + B)
+int64_t bwd_capacity(int32_t B, int32_t H, int32_t total) {
+  return static_cast<int64_t>(H) * (total / kTileRows + B);
+}
+
+int64_t bwd_plan_bytes(int32_t B, int32_t H, int32_t total) {
+  return 32 + static_cast<int64_t>(pad16(static_cast<size_t>(B) + 1)) + 2 * bwd_capacity(B, H, total) * 16;
+}
+
+// Both backward kernels over a plan written by bwd_schedule_kernel.  Arguments already checked.
+template <int D, bool kDQ>
+cudaError_t launch_bwd_kernel(const CUtensorMap& f0, const CUtensorMap& f1, const CUtensorMap& s0,
+                              const CUtensorMap& s1, const BwdParams& p, int grid, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kBwdThreads);
+  cfg.dynamicSmemBytes = BwdCfg<D>::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, hstu_bwd_kernel<D, kDQ>, f0, f1, s0, s1, p);
+}
+
+template <int D>
+cudaError_t launch_bwd_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, BwdParams pkv, BwdParams pq, int grid_kv, int grid_q,
+                            cudaStream_t stream) {
+  cudaError_t e = launch_bwd_kernel<D, false>(tk, tv, tq, tdo, pkv, grid_kv, stream);
+  if (e == cudaSuccess) e = launch_bwd_kernel<D, true>(tq, tdo, tk, tv, pq, grid_q, stream);
+  return e;
+}
+
+hstu_status_t run_bwd(const void* q, const void* k, const void* v, const void* dout, const int32_t* seq_offsets,
+                      const int32_t* num_targets, int32_t B, int32_t H, int32_t d, int32_t total,
+                      int32_t max_seq_len, float alpha, float N, void* dq, void* dk, void* dv, void* stream_ptr) {
+  if (B < 0 || H < 1 || total < 0 || max_seq_len < 0) return HSTU_ERR_INVALID_ARGUMENT;
+  if (bwd_capacity(B, H, total) > INT_MAX / 2) return HSTU_ERR_UNSUPPORTED;
+  // q, k, v, dq share the checks of a forward call (dq in the role of out), then the other
+  // gradients must not overlap any input or each other.
+  hstu_status_t s = check_tokens(q, k, v, seq_offsets, H, d, total, total, alpha, N, dq);
+  if (s != HSTU_OK) return s;
+  if (total == 0 || B == 0) return HSTU_OK;
+  if (!dout || !dk || !dv) return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(dout) || !aligned16(dk) || !aligned16(dv)) return HSTU_ERR_UNSUPPORTED;
+  const size_t bytes = static_cast<size_t>(total) * H * d * 2;
+  const void* ins[4] = {q, k, v, dout};
+  void* outs[3] = {dq, dk, dv};
+  for (int o = 0; o < 3; ++o) {
+    for (int i = 0; i < 4; ++i)
+      if (overlaps(outs[o], bytes, ins[i], bytes)) return HSTU_ERR_INVALID_ARGUMENT;
+    for (int o2 = o + 1; o2 < 3; ++o2)
+      if (overlaps(outs[o], bytes, outs[o2], bytes)) return HSTU_ERR_INVALID_ARGUMENT;
+  }
+  DeviceState* st = device_state();
+  if (!st || !encoder()) return HSTU_ERR_CUDA;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  const int64_t row_elems = static_cast<int64_t>(H) * d;
+  CUtensorMap tq, tk, tv, tdo;
+  const uint32_t box_x = d >= 64 ? 64u : 32u;
+  const CUtensorMapSwizzle swz = d >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!encode_rows(&tq, q, total, row_elems, box_x, swz) || !encode_rows(&tk, k, total, row_elems, box_x, swz) ||
+      !encode_rows(&tv, v, total, row_elems, box_x, swz) || !encode_rows(&tdo, dout, total, row_elems, box_x, swz))
+    return HSTU_ERR_CUDA;
+  void* plan = nullptr;
+  if (cudaMallocFromPoolAsync(&plan, static_cast<size_t>(bwd_plan_bytes(B, H, total)), st->pool, stream) !=
+      cudaSuccess)
+    return HSTU_ERR_CUDA;
+  uint8_t* pb = static_cast<uint8_t*>(plan);
+  int32_t* header = reinterpret_cast<int32_t*>(pb);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(pb + 32);
+  const int64_t cap = bwd_capacity(B, H, total);
+  int4* dq_items = reinterpret_cast<int4*>(pb + 32 + pad16(static_cast<size_t>(B) + 1));
+  int4* kv_items = dq_items + cap;
+  BwdSchedArgs a;
+  a.seq_offsets = seq_offsets;
+  a.num_targets = num_targets;
+  a.B = B;
+  a.H = H;
+  a.total = total;
+  a.max_seq_len = max_seq_len;
+  a.nbins = cost_bins(max_seq_len);
+  a.max_items = static_cast<int32_t>(cap);
+  a.header = header;
+  a.tile_start = tile_start;
+  a.dq_items = dq_items;
+  a.kv_items = kv_items;
+  a.err = st->err_word;
+  bwd_schedule_kernel<<<1, kSchedThreads, 0, stream>>>(a);
+  s = cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  if (s == HSTU_OK) {
+    BwdParams pkv;
+    pkv.seq_offsets = seq_offsets;
+    pkv.num_targets = num_targets;
+    pkv.items = kv_items;
+    pkv.num_items = header + 5;
+    pkv.work_counter = header + 4;
+    pkv.done_counter = header + 6;
+    pkv.out0 = static_cast<__nv_bfloat16*>(dv);
+    pkv.out1 = static_cast<__nv_bfloat16*>(dk);
+    pkv.H = H;
+    pkv.half_alpha = 0.5f * alpha;
+    pkv.ds_scale = 0.5f * alpha / N;
+    pkv.inv_n = 1.0f / N;
+    pkv.err = st->err_word;
+    BwdParams pq = pkv;
+    pq.items = dq_items;
+    pq.num_items = header + 1;
+    pq.work_counter = header + 0;
+    pq.done_counter = header + 2;
+    pq.out0 = static_cast<__nv_bfloat16*>(dq);
+    pq.out1 = nullptr;
+    const int grid = static_cast<int>(cap < st->num_sms ? cap : st->num_sms);
+    cudaError_t e;
+    if (d == 128) e = launch_bwd_pair<128>(tq, tk, tv, tdo, pkv, pq, grid, grid, stream);
+    else if (d == 64) e = launch_bwd_pair<64>(tq, tk, tv, tdo, pkv, pq, grid, grid, stream);
+    else e = launch_bwd_pair<32>(tq, tk, tv, tdo, pkv, pq, grid, grid, stream);
+    if (e != cudaSuccess) s = HSTU_ERR_CUDA;
+  }
+  if (cudaFreeAsync(plan, stream) != cudaSuccess && s == HSTU_OK) s = HSTU_ERR_CUDA;
+  return s;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------------------------
@@ -379,6 +516,14 @@ hstu_status_t hstu_attn_fwd_rab(const void* q, const void* k, const void* v, con
   if (rab && (reinterpret_cast<uintptr_t>(rab) & 3u)) return HSTU_ERR_UNSUPPORTED;
   return hstu::run(q, k, v, seq_offsets, num_targets, cached_len, B, H, d, total_kv, total_q, max_seq_len, alpha,
                    N, out, stream, rab, rab_len);
+}
+
+hstu_status_t hstu_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
+                            const int32_t* seq_offsets, const int32_t* num_targets, int32_t B, int32_t H, int32_t d,
+                            int32_t total_tokens, int32_t max_seq_len, float alpha, float N, void* dq, void* dk,
+                            void* dv, void* stream) {
+  return hstu::run_bwd(q, k, v, dout, seq_offsets, num_targets, B, H, d, total_tokens, max_seq_len, alpha, N, dq,
+                       dk, dv, stream);
 }
 
 int64_t hstu_attn_plan_bytes(int32_t B, int32_t H, int32_t total_q) {
@@ -463,6 +608,58 @@ hstu_status_t hstu_attn_gemm_bf16(const void* a, const void* w, void* c, int32_t
   hstu::gemm_bf16_kernel<<<grid, hstu::kGemmThreads, hstu::GemmCfg::kSmemBytes,
                            static_cast<cudaStream_t>(stream_ptr)>>>(ta, tw, p);
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status_t hstu_attn_partition(const int32_t* seq_offsets, const int32_t* num_targets,
+                                  const int32_t* cached_len, int32_t B, int32_t parts, int32_t* user_start) {
+  if (B < 0 || parts < 1 || !user_start || (B > 0 && !seq_offsets)) return HSTU_ERR_INVALID_ARGUMENT;
+  // Cost of user b: its visible (query, key) pairs, sum over queried positions i in [c, L) of
+  // |A(i)| = i + 1 (history, i < U) or U + 1 (candidate).
+  std::vector<int64_t> cost(static_cast<size_t>(B));
+  int64_t total = 0, largest = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    const int64_t L = static_cast<int64_t>(seq_offsets[b + 1]) - seq_offsets[b];
+    const int64_t T = num_targets ? num_targets[b] : 0;
+    const int64_t c = cached_len ? cached_len[b] : 0;
+    if (L < 0 || T < 0 || T > L || c < 0 || c > L - T) return HSTU_ERR_BAD_OFFSETS;
+    const int64_t U = L - T;
+    const int64_t hist = c < U ? (U * (U + 1) - c * (c + 1)) / 2 : 0;
+    cost[b] = hist + (L - (U > c ? U : c)) * (U + 1);
+    total += cost[b];
+    largest = cost[b] > largest ? cost[b] : largest;
+  }
+  // Smallest cap such that consecutive users fill at most `parts` parts of cost <= cap.
+  auto parts_needed = [&](int64_t cap) {
+    int32_t n = 1;
+    int64_t run = 0;
+    for (int32_t b = 0; b < B; ++b) {
+      if (run + cost[b] > cap) {
+        ++n;
+        run = 0;
+      }
+      run += cost[b];
+    }
+    return n;
+  };
+  int64_t lo = largest, hi = total > largest ? total : largest;
+  while (lo < hi) {
+    const int64_t mid = lo + (hi - lo) / 2;
+    if (parts_needed(mid) <= parts) hi = mid;
+    else lo = mid + 1;
+  }
+  // Fill parts left to right under that cap; parts left over at the end are empty.
+  int32_t part = 0;
+  int64_t run = 0;
+  user_start[0] = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    if (run + cost[b] > lo && run > 0 && part + 1 < parts) {
+      user_start[++part] = b;
+      run = 0;
+    }
+    run += cost[b];
+  }
+  for (int32_t k = part + 1; k <= parts; ++k) user_start[k] = B;
+  return HSTU_OK;
 }
 
 hstu_status_t hstu_attn_selfcheck_wait_timeout(uint64_t limit_ns, void* stream_ptr) {

@@ -1,0 +1,490 @@
+// hstu_bwd_sm100.cuh — backward pass of jagged target-aware HSTU pointwise attention for sm_100a.
+//
+// Forward (DLRMv3 review, section "model selection"): out = Mask(SiLU(alpha Q K^T)) V / N.  The
+// pages print no backward pass; by the chain rule, with dO the loss gradient of out and for every
+// visible pair (i, j):
+//   x = alpha q_i.k_j,  p = silu(x),  g = dO_i.v_j / N,  ds = g silu'(x) alpha
+//   dV_j += p dO_i / N,  dQ_i += ds k_j,  dK_j += ds q_i
+// With h = x/2 and t = tanh(h):  p = h (1 + t),  silu'(x) = (1 + t)(1 + h - h t) / 2, so one
+// tanh.approx.f32 per pair gives both p and silu'.
+//
+// hstu_bwd_kernel<D, kDQ> is one persistent kernel body for both halves of the work:
+//   kDQ = false (dK/dV): an item owns one 128-key tile; its K and V tiles stay in shared memory
+//       ("fixed" pair) while the query tiles that see it stream through a ring (Q and dO).
+//         S^T = K Q^T, dP^T = V dO^T                      (SS MMAs into TMEM)
+//         P^T, dS^T in registers (thread = key row)        -> bf16 into TMEM over S^T, dP^T
+//         dV += P^T dO, dK += dS^T Q                       (TS MMAs, P^T / dS^T read from TMEM)
+//   kDQ = true (dQ): an item owns one 128-query tile; Q and dO stay, K and V stream.
+//         S = Q K^T, dP = dO V^T;  dS (thread = query row);  dQ += dS K
+// No atomics: every output row is written once, by the item that owns it.
+//
+//   warp 8      producer: fetches the next item, TMA-loads the fixed pair and streams the pairs
+//   warp 9      MMA issuer (lane 0 issues, the warp runs converged)
+//   warps 0-7   elementwise + epilogue: warp w owns TMEM lane quarter w % 4 and score columns
+//               [64 (w / 4), 64 (w / 4) + 64); its bf16 results overwrite the first half of its
+//               own column range, so no warp writes a column another warp still has to read.
+//
+// TMEM columns: S [0,128), dP [128,256), accumulator 0 [256, 256+D), accumulator 1 [256+D, 256+2D)
+// (dK/dV: acc0 = dV, acc1 = dK;  dQ: acc0 = dQ).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "bwd_schedule.cuh"
+#include "hstu_fwd_sm100.cuh"
+#include "sm100_ptx.cuh"
+
+namespace hstu {
+
+template <int D>
+struct BwdCfg {
+  using T = FwdCfg<D>;  // tile geometry: swizzle, column blocks, bytes per 128-row tile
+  static constexpr int kStages = (D == 128) ? 2 : 4;  // ring stages; each holds a pair of tiles
+  static constexpr int kSmemTiles = (2 + 2 * kStages) * T::kTileBytes;
+  static constexpr int kSmemBytes = 1024 + kSmemTiles + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColA0 = 256, kColA1 = 256 + D;
+  static constexpr uint32_t kIdescScore = ptx::idesc_bf16_f32(128, 128, false);
+  static constexpr uint32_t kIdescAcc = ptx::idesc_bf16_f32(128, D, true);
+};
+
+constexpr int kBwdThreads = 320;
+
+struct BwdParams {
+  const int32_t* seq_offsets;
+  const int32_t* num_targets;  // may be null
+  const int4* items;
+  const int32_t* num_items;
+  int32_t* work_counter;
+  int32_t* done_counter;
+  __nv_bfloat16* out0;  // dK/dV: dV;  dQ: dQ
+  __nv_bfloat16* out1;  // dK/dV: dK;  dQ: unused
+  int32_t H;
+  float half_alpha;     // alpha / 2
+  float ds_scale;       // alpha / (2 N)
+  float inv_n;
+  unsigned* err;
+};
+
+template <int kStages>
+struct BwdCtl {
+  uint64_t fix_full, fix_empty;
+  uint64_t ring_full[kStages], ring_empty[kStages];
+  uint64_t s_full, p_full, o_full, o_empty;
+  uint64_t sched_full[2], sched_empty[2];
+  uint64_t drain;
+  // work slot: valid, h, row0 (first token row of the user), fixed tile, L, U, e1, s2, e2
+  int32_t slot[2][10];
+  uint32_t tmem_base;
+  int32_t abort_flag;
+};
+
+struct BwdWork {
+  int valid, h, row0, fixed, L, U;
+  TileRange r;
+};
+
+__device__ __forceinline__ BwdWork read_bwd_slot(const volatile int32_t* s) {
+  BwdWork w;
+  w.valid = s[0];
+  w.h = s[1];
+  w.row0 = s[2];
+  w.fixed = s[3];
+  w.L = s[4];
+  w.U = s[5];
+  w.r.e1 = s[6];
+  w.r.s2 = s[7];
+  w.r.e2 = s[8];
+  return w;
+}
+
+// 32 score columns of this thread's row: S and dP chunks in registers -> dS (and, for dK/dV, P)
+// packed as bf16 pairs into 16 TMEM columns each.  The visible columns are [lo, hi) plus `self`
+// (relative to the chunk's first column), everything else is an exact zero.
+template <bool kDQ>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], uint32_t t_p,
+                                          uint32_t t_ds, float half_alpha, float ds_scale, bool full, int lo, int hi,
+                                          int self) {
+  uint32_t pk_p[16], pk_ds[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    float p2[2], d2[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int c = 2 * e + u;
+      const float h = __uint_as_float(s[c]) * half_alpha;
+      const float t = ptx::tanh_approx(h);
+      const float a = 1.0f + t;
+      const float w = fmaf(-h, t, h) + 1.0f;
+      float ds = __uint_as_float(dp[c]) * ds_scale * a * w;
+      float p = h * a;
+      if (!full) {
+        const bool vis = (c >= lo && c < hi) || c == self;
+        ds = vis ? ds : 0.0f;
+        p = vis ? p : 0.0f;
+      }
+      p2[u] = p;
+      d2[u] = ds;
+    }
+    pk_ds[e] = pack_bf16x2(d2[0], d2[1]);
+    if constexpr (!kDQ) pk_p[e] = pack_bf16x2(p2[0], p2[1]);
+  }
+  ptx::tmem_st16(t_ds, pk_ds);
+  if constexpr (!kDQ) ptx::tmem_st16(t_p, pk_p);
+}
+
+template <int D, bool kDQ>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    hstu_bwd_kernel(const __grid_constant__ CUtensorMap tm_f0, const __grid_constant__ CUtensorMap tm_f1,
+                    const __grid_constant__ CUtensorMap tm_s0, const __grid_constant__ CUtensorMap tm_s1,
+                    const BwdParams p) {
+  using Cfg = BwdCfg<D>;
+  using T = typename Cfg::T;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw_addr = ptx::smem_addr(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  const uint32_t sbase = ptx::smem_addr(smem);
+  const uint32_t sFix = sbase;                          // 2 tiles: fixed[0], fixed[1]
+  const uint32_t sRing = sbase + 2 * T::kTileBytes;     // kStages x 2 tiles
+  auto* ctl = reinterpret_cast<BwdCtl<Cfg::kStages>*>(smem + Cfg::kSmemTiles);
+  volatile int32_t* abort_flag = &ctl->abort_flag;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  auto bar = [](const uint64_t& b) { return ptx::smem_addr(&b); };
+
+  if (warp == kProducerWarp && lane == 0) {
+    ptx::mbar_init(bar(ctl->fix_full), 1);
+    ptx::mbar_init(bar(ctl->fix_empty), 1);
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      ptx::mbar_init(bar(ctl->ring_full[s]), 1);
+      ptx::mbar_init(bar(ctl->ring_empty[s]), 1);
+    }
+    ptx::mbar_init(bar(ctl->s_full), 1);
+    ptx::mbar_init(bar(ctl->p_full), 8);
+    ptx::mbar_init(bar(ctl->o_full), 1);
+    ptx::mbar_init(bar(ctl->o_empty), 8);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar(ctl->sched_full[i]), 1);
+      ptx::mbar_init(bar(ctl->sched_empty[i]), 1 + 8);
+    }
+    ptx::mbar_init(bar(ctl->drain), 1);
+    ctl->abort_flag = 0;
+    ptx::fence_mbarrier_init();
+    ptx::prefetch_tmap(&tm_f0);
+    ptx::prefetch_tmap(&tm_f1);
+    ptx::prefetch_tmap(&tm_s0);
+    ptx::prefetch_tmap(&tm_s1);
+  }
+  if (warp == kMmaWarp) {
+    ptx::tmem_alloc(ptx::smem_addr(&ctl->tmem_base), Cfg::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      const int M = *p.num_items;
+      int slot = 0;
+      uint32_t sched_empty_par[2] = {1u, 1u};
+      uint32_t fix_empty_par = 1u;
+      int stage = 0;
+      uint32_t ring_phase = 0;
+      bool ok = true;
+      int issued_fix = 0, issued_ring = 0;
+      while (ok) {
+        const int idx = atomicAdd(p.work_counter, 1);
+        BwdWork w{};
+        w.valid = idx < M;
+        if (w.valid) {
+          const int4 it = p.items[idx];
+          const int b = it.x;
+          w.fixed = it.y;
+          w.h = it.z;
+          w.row0 = p.seq_offsets[b];
+          w.L = p.seq_offsets[b + 1] - w.row0;
+          w.U = w.L - (p.num_targets ? p.num_targets[b] : 0);
+          w.r = kDQ ? key_tiles_of_query_tile(w.fixed, w.L, w.U) : query_tiles_of_key_tile(w.fixed, w.L, w.U);
+        }
+        if (!wait_bounded(bar(ctl->sched_empty[slot]), sched_empty_par[slot], abort_flag, p.err)) break;
+        sched_empty_par[slot] ^= 1u;
+        volatile int32_t* s = ctl->slot[slot];
+        s[0] = w.valid; s[1] = w.h; s[2] = w.row0; s[3] = w.fixed; s[4] = w.L; s[5] = w.U;
+        s[6] = w.r.e1; s[7] = w.r.s2; s[8] = w.r.e2;
+        ptx::mbar_arrive(bar(ctl->sched_full[slot]));
+        slot ^= 1;
+        if (!w.valid) break;
+
+        const int col = w.h * D;
+        if (!wait_bounded(bar(ctl->fix_empty), fix_empty_par, abort_flag, p.err)) break;
+        fix_empty_par ^= 1u;
+        ptx::mbar_arrive_expect_tx(bar(ctl->fix_full), 2 * T::kTileBytes);
+        for (int blk = 0; blk < T::kBlocks; ++blk) {
+          const int row = w.row0 + w.fixed * kTileRows;
+          ptx::tma_load_2d(sFix + blk * T::kBlockBytes, &tm_f0, bar(ctl->fix_full), col + blk * T::kBlockElems, row);
+          ptx::tma_load_2d(sFix + T::kTileBytes + blk * T::kBlockBytes, &tm_f1, bar(ctl->fix_full),
+                           col + blk * T::kBlockElems, row);
+        }
+        ++issued_fix;
+        const int n = tile_count(w.r);
+        for (int i = 0; i < n; ++i) {
+          if (!wait_bounded(bar(ctl->ring_empty[stage]), ring_phase ^ 1u, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar(ctl->ring_full[stage]);
+          ptx::mbar_arrive_expect_tx(fb, 2 * T::kTileBytes);
+          const int row = w.row0 + tile_at(w.r, i) * kTileRows;
+          const uint32_t dst = sRing + stage * 2 * T::kTileBytes;
+          for (int blk = 0; blk < T::kBlocks; ++blk) {
+            ptx::tma_load_2d(dst + blk * T::kBlockBytes, &tm_s0, fb, col + blk * T::kBlockElems, row);
+            ptx::tma_load_2d(dst + T::kTileBytes + blk * T::kBlockBytes, &tm_s1, fb, col + blk * T::kBlockElems, row);
+          }
+          ++issued_ring;
+          if (++stage == Cfg::kStages) {
+            stage = 0;
+            ring_phase ^= 1u;
+          }
+        }
+      }
+      if (*abort_flag) {
+        // Let every copy this CTA started land before its shared memory is released.
+        for (int k = 1; k <= Cfg::kStages && k <= issued_ring; ++k) {
+          const int pos = issued_ring - k;
+          drain_wait(bar(ctl->ring_full[pos % Cfg::kStages]), (uint32_t)((pos / Cfg::kStages) & 1));
+        }
+        if (issued_fix > 0) drain_wait(bar(ctl->fix_full), (uint32_t)((issued_fix - 1) & 1));
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    const uint32_t lead = (lane == 0) ? 1u : 0u;
+    auto wait_all = [&](uint32_t b, uint32_t par) {
+      return __all_sync(0xffffffffu, wait_bounded(b, par, abort_flag, p.err));
+    };
+    const uint64_t dfix = ptx::smem_desc(sFix, 16, 8 * T::kRowBytes, T::kSwizzle);       // K-major A
+    const uint64_t dring = ptx::smem_desc(sRing, 16, 8 * T::kRowBytes, T::kSwizzle);     // K-major B
+    const uint64_t dringmn = ptx::smem_desc(sRing, T::kBlockBytes, 8 * T::kRowBytes, T::kSwizzle);  // MN-major B
+    int slot = 0;
+    uint32_t sched_full_par[2] = {0u, 0u};
+    uint32_t fix_full_par = 0u, p_full_par = 0u, o_empty_par = 1u;
+    int stage = 0;
+    uint32_t ring_phase = 0;
+    bool ok = true;
+    // Accumulating MMAs of streamed tile `st` (ring stage `sst`), whose P / dS are in TMEM.
+    auto accumulate = [&](int sst, bool first) {
+      const uint64_t base_mn = dringmn + ((sst * 2 * T::kTileBytes) >> 4);
+#pragma unroll
+      for (int ks = 0; ks < kTileRows / 16; ++ks) {
+        const uint32_t acol = 64 * (ks >> 2) + 8 * (ks & 3);
+        const uint32_t acc = (first && ks == 0) ? 0u : 1u;
+        const uint64_t boff = (ks * 16 * T::kRowBytes) >> 4;
+        if constexpr (kDQ) {
+          // dQ += dS K: dS from the dP columns, K = streamed tile 0.
+          ptx::mma_ts_lead(lead, tmem + Cfg::kColA0, tmem + Cfg::kColDP + acol, base_mn + boff, Cfg::kIdescAcc, acc);
+        } else {
+          // dV += P^T dO (dO = streamed tile 1), dK += dS^T Q (Q = streamed tile 0).
+          ptx::mma_ts_lead(lead, tmem + Cfg::kColA0, tmem + Cfg::kColS + acol,
+                           base_mn + ((T::kTileBytes) >> 4) + boff, Cfg::kIdescAcc, acc);
+          ptx::mma_ts_lead(lead, tmem + Cfg::kColA1, tmem + Cfg::kColDP + acol, base_mn + boff, Cfg::kIdescAcc, acc);
+        }
+      }
+    };
+    while (ok) {
+      if (!wait_all(bar(ctl->sched_full[slot]), sched_full_par[slot])) break;
+      sched_full_par[slot] ^= 1u;
+      const BwdWork w = read_bwd_slot(ctl->slot[slot]);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(ctl->sched_empty[slot]));
+      slot ^= 1;
+      if (!w.valid) break;
+      const int n = tile_count(w.r);
+      if (!wait_all(bar(ctl->fix_full), fix_full_par)) break;
+      fix_full_par ^= 1u;
+      ptx::tc_fence_after();
+      int prev_stage = 0;
+      for (int i = 0; i <= n && ok; ++i) {
+        if (i > 0) {
+          // The previous tile's P / dS are in TMEM: accumulate, then free its ring stage.
+          ok = wait_all(bar(ctl->p_full), p_full_par) && (i > 1 || wait_all(bar(ctl->o_empty), o_empty_par));
+          if (!ok) break;
+          p_full_par ^= 1u;
+          if (i == 1) o_empty_par ^= 1u;
+          ptx::tc_fence_after();
+          accumulate(prev_stage, i == 1);
+          ptx::mma_commit_lead(lead, bar(ctl->ring_empty[prev_stage]));
+        }
+        if (i < n) {
+          if (!wait_all(bar(ctl->ring_full[stage]), ring_phase)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint64_t ds0 = dring + ((stage * 2 * T::kTileBytes) >> 4);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (ks / T::kKStepsPerBlock) * T::kBlockBytes + (ks % T::kKStepsPerBlock) * 32;
+            // scores: fixed[0] x streamed[0]^T -> S;  fixed[1] x streamed[1]^T -> dP
+            ptx::mma_ss_lead(lead, tmem + Cfg::kColS, dfix + (off >> 4), ds0 + (off >> 4), Cfg::kIdescScore,
+                             ks > 0 ? 1u : 0u);
+            ptx::mma_ss_lead(lead, tmem + Cfg::kColDP, dfix + ((T::kTileBytes + off) >> 4),
+                             ds0 + ((T::kTileBytes + off) >> 4), Cfg::kIdescScore, ks > 0 ? 1u : 0u);
+          }
+          ptx::mma_commit_lead(lead, bar(ctl->s_full));
+          prev_stage = stage;
+          if (++stage == Cfg::kStages) {
+            stage = 0;
+            ring_phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) break;
+      ptx::mma_commit_lead(lead, bar(ctl->fix_empty));  // fixed pair free after the item's last MMA
+      ptx::mma_commit_lead(lead, bar(ctl->o_full));     // accumulators complete
+    }
+    ptx::mma_commit_lead(lead, bar(ctl->drain));
+    drain_wait(bar(ctl->drain), 0u);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ elementwise + epilogue
+    const int quarter = warp & 3;
+    const int ch = warp >> 2;                      // score columns [64 ch, 64 ch + 64)
+    const int row = quarter * 32 + lane;           // row of the fixed tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + Cfg::kColS + 64 * ch;
+    const uint32_t t_dp = tmem + lane_off + Cfg::kColDP + 64 * ch;
+    int slot = 0;
+    uint32_t sched_full_par[2] = {0u, 0u};
+    uint32_t s_full_par = 0u, o_full_par = 0u;
+    bool ok = true;
+    while (ok) {
+      ok = __all_sync(0xffffffffu, wait_bounded(bar(ctl->sched_full[slot]), sched_full_par[slot], abort_flag, p.err));
+      if (!ok) break;
+      sched_full_par[slot] ^= 1u;
+      const BwdWork w = read_bwd_slot(ctl->slot[slot]);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(ctl->sched_empty[slot]));
+      slot ^= 1;
+      if (!w.valid) break;
+      const int n = tile_count(w.r);
+      const int pos = w.fixed * kTileRows + row;  // this thread's position in the segment
+      for (int i = 0; i < n; ++i) {
+        const int c0 = tile_at(w.r, i) * kTileRows + 64 * ch;  // position of this warp's first column
+        ok = __all_sync(0xffffffffu, wait_bounded(bar(ctl->s_full), s_full_par, abort_flag, p.err));
+        if (!ok) break;
+        s_full_par ^= 1u;
+        ptx::tc_fence_after();
+        // Visible columns, relative to c0: [lo, hi) plus self.
+        int lo, hi, self;
+        bool full;
+        if constexpr (kDQ) {
+          // query `pos` sees keys [0, min(pos + 1, U)) and itself
+          lo = -c0;
+          hi = (pos < w.U ? pos + 1 : w.U) - c0;
+          self = pos - c0;
+          full = (c0 + 64 <= w.U) && (c0 + 64 <= pos + 1) && pos < w.L;
+        } else {
+          // key `pos` is seen by queries [pos, L) if it is history, by itself alone otherwise
+          lo = pos - c0;
+          hi = (pos < w.U ? w.L : pos + 1) - c0;
+          if (pos >= w.L) hi = lo;
+          self = -1;
+          full = (lo <= 0) && (hi >= 64);
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          uint32_t rs[32], rd[32];
+          ptx::tmem_ld32(t_s + 32 * k, rs);
+          ptx::tmem_ld32(t_dp + 32 * k, rd);
+          ptx::tmem_ld_wait(rs);
+          ptx::tmem_ld_wait(rd);
+          bwd_chunk<kDQ>(rs, rd, t_s + 16 * k, t_dp + 16 * k, p.half_alpha, p.ds_scale, full, lo - 32 * k,
+                         hi - 32 * k, self - 32 * k);
+        }
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(ctl->p_full));
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, wait_bounded(bar(ctl->o_full), o_full_par, abort_flag, p.err));
+      if (!ok) break;
+      o_full_par ^= 1u;
+      ptx::tc_fence_after();
+      // Epilogue: rows of the fixed tile that exist.  dK/dV: warps of column half 0 write dV
+      // (scaled by 1/N), half 1 writes dK.  dQ: the two halves split dQ's columns.
+      const bool live = w.fixed * kTileRows + row < w.L;
+      const size_t grow = (size_t)(w.row0 + w.fixed * kTileRows + row);
+      if constexpr (kDQ) {
+        constexpr int kPer = (D / 32 + 1) / 2;  // 32-column chunks per warp
+#pragma unroll
+        for (int c = 0; c < kPer; ++c) {
+          const int cc = ch * kPer + c;
+          if (cc < D / 32) {
+            uint32_t ro[32];
+            ptx::tmem_ld32(tmem + lane_off + Cfg::kColA0 + 32 * cc, ro);
+            ptx::tmem_ld_wait(ro);
+            if (live) {
+              uint4* d4 = reinterpret_cast<uint4*>(p.out0 + (grow * p.H + w.h) * D + 32 * cc);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 0]), __uint_as_float(ro[q4 * 8 + 1]));
+                v.y = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 2]), __uint_as_float(ro[q4 * 8 + 3]));
+                v.z = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 4]), __uint_as_float(ro[q4 * 8 + 5]));
+                v.w = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 6]), __uint_as_float(ro[q4 * 8 + 7]));
+                d4[q4] = v;
+              }
+            }
+          }
+        }
+      } else {
+        const uint32_t col = ch ? Cfg::kColA1 : Cfg::kColA0;
+        const float scale = ch ? 1.0f : p.inv_n;
+        __nv_bfloat16* dst = (ch ? p.out1 : p.out0) + (grow * p.H + w.h) * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ro[32];
+          ptx::tmem_ld32(tmem + lane_off + col + 32 * cc, ro);
+          ptx::tmem_ld_wait(ro);
+          if (live) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cc);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 0]) * scale, __uint_as_float(ro[q4 * 8 + 1]) * scale);
+              v.y = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 2]) * scale, __uint_as_float(ro[q4 * 8 + 3]) * scale);
+              v.z = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 4]) * scale, __uint_as_float(ro[q4 * 8 + 5]) * scale);
+              v.w = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 6]) * scale, __uint_as_float(ro[q4 * 8 + 7]) * scale);
+              d4[q4] = v;
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(ctl->o_empty));
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.done_counter, 1) == (int)gridDim.x - 1) {
+      atomicExch(p.work_counter, 0);
+      atomicExch(p.done_counter, 0);
+    }
+  }
+}
+
+}  // namespace hstu

@@ -89,8 +89,51 @@ struct SchedArgs {
   unsigned* err;          // device error word
 };
 
+// Inclusive block-wide prefix sums of two values per thread (kSchedThreads threads); also
+// returns the block totals.  `scratch` holds 2 x 32 values.
+__device__ __forceinline__ void block_inclusive_scan2(long long& a, long long& b, long long (*scratch)[32],
+                                                      long long& total_a, long long& total_b) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long na = __shfl_up_sync(0xffffffffu, a, o);
+    const long long nb = __shfl_up_sync(0xffffffffu, b, o);
+    if (lane >= o) {
+      a += na;
+      b += nb;
+    }
+  }
+  if (lane == 31) {
+    scratch[0][warp] = a;
+    scratch[1][warp] = b;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    long long wa = scratch[0][lane], wb = scratch[1][lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long na = __shfl_up_sync(0xffffffffu, wa, o);
+      const long long nb = __shfl_up_sync(0xffffffffu, wb, o);
+      if (lane >= o) {
+        wa += na;
+        wb += nb;
+      }
+    }
+    scratch[0][lane] = wa;
+    scratch[1][lane] = wb;
+  }
+  __syncthreads();
+  if (warp > 0) {
+    a += scratch[0][warp - 1];
+    b += scratch[1][warp - 1];
+  }
+  total_a = scratch[0][31];
+  total_b = scratch[1][31];
+  __syncthreads();
+}
+
 // Inclusive block-wide prefix sum of one value per thread (kSchedThreads threads); also
-// returns the block total.  `scratch` holds 32 ints.
+// returns the block total.  `scratch` holds 32 values.
 __device__ __forceinline__ long long block_inclusive_scan(long long v, long long* scratch,
                                                           long long* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -136,7 +179,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
   // (griddepcontrol.wait) before it reads anything in global memory.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ int hist[kMaxCostBins];
-  __shared__ long long scan_scratch[32];
+  __shared__ long long scan_scratch[2][32];
   __shared__ long long carry_q, carry_p;
   // Per-user values of pass 1, kept on chip for passes 2 and 4 when the batch is small enough
   // (their reads are then shared-memory latency instead of a chain of global loads).
@@ -150,53 +193,57 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
   if (tid == 0) {
     carry_q = 0;
     carry_p = 0;
-    if (a.seq_offsets[0] != 0 || a.seq_offsets[a.B] != a.total_kv) atomicOr(a.err, kErrBadOffsets);
   }
   __syncthreads();
 
   // Pass 1: per-user validation; one scan gives both the query-row starts (the caller's layout)
-  // and the block starts.
+  // and the block starts.  Lengths are taken in 64 bits, so that corrupt offsets cannot wrap.
   for (int base = 0; base < a.B; base += kSchedThreads) {
     const int b = base + tid;
     long long nq = 0, npairs = 0;  // rows in the layout; 256-row blocks to compute
     bool ok = false;
+    int L = 0, T = 0, c = 0;
     if (b < a.B) {
       const int o0 = a.seq_offsets[b], o1 = a.seq_offsets[b + 1];
-      const int L = o1 - o0;
-      const int T = a.num_targets ? a.num_targets[b] : 0;
-      const int c = a.cached_len ? a.cached_len[b] : 0;
-      ok = o0 >= 0 && L >= 0 && o1 <= a.total_kv && L <= a.max_seq_len && T >= 0 && T <= L && c >= 0 &&
-           c <= L - T;
+      const long long L64 = (long long)o1 - o0;
+      T = a.num_targets ? a.num_targets[b] : 0;
+      c = a.cached_len ? a.cached_len[b] : 0;
+      ok = o0 >= 0 && L64 >= 0 && o1 <= a.total_kv && L64 <= a.max_seq_len && T >= 0 && T <= L64 && c >= 0 &&
+           c <= L64 - T;
+      if (b == 0 && o0 != 0) ok = false;
+      if (b == a.B - 1 && o1 != a.total_kv) ok = false;
       if (!ok) atomicOr(a.err, kErrBadOffsets);
-      // A skipped user still owns its rows of the layout, so later users keep their places.
-      const int cc = c < 0 ? 0 : c;
-      nq = L > cc ? (long long)(L - cc) : 0;
+      L = ok ? (int)L64 : 0;
+      // A skipped user still owns its rows of the layout, so later users keep their places; a
+      // corrupt length is capped, and the layout check below then skips what follows it.
+      const long long cc = c < 0 ? 0 : c;
+      nq = L64 > cc ? L64 - cc : 0;
+      if (nq > (long long)a.total_q + 1) nq = (long long)a.total_q + 1;
       npairs = ok ? cdiv(L - c, kPairRows) : 0;
     }
-    long long tot;
-    const long long incl = block_inclusive_scan((nq << 32) | npairs, scan_scratch, &tot);
-    const long long start_q = carry_q + (incl >> 32) - nq;
-    const long long start_p = carry_p + (incl & 0xffffffffll) - npairs;
+    long long incl_q = nq, incl_p = npairs, tot_q, tot_p;
+    block_inclusive_scan2(incl_q, incl_p, scan_scratch, tot_q, tot_p);
+    const long long start_q = carry_q + incl_q - nq;
+    const long long start_p = carry_p + incl_p - npairs;
     if (b < a.B) {
-      if (ok && start_q + nq > a.total_q) {
+      if (ok && (start_q < 0 || start_q + nq > a.total_q)) {
         ok = false;
         atomicOr(a.err, kErrBadOffsets);
       }
       a.q_start[b] = ok ? (int)start_q : -1;
       a.pair_start[b] = (int)start_p;
       if (cached) {
-        const int o0 = a.seq_offsets[b], L = a.seq_offsets[b + 1] - o0;
         s_L[b] = L;
-        s_U[b] = L - (a.num_targets ? a.num_targets[b] : 0);
-        s_c[b] = a.cached_len ? a.cached_len[b] : 0;
+        s_U[b] = L - T;
+        s_c[b] = c;
         s_q[b] = ok ? (int)start_q : -1;
         s_ps[b] = (int)start_p;
       }
     }
     __syncthreads();
     if (tid == 0) {
-      carry_q += tot >> 32;
-      carry_p += tot & 0xffffffffll;
+      carry_q += tot_q;
+      carry_p += tot_p;
     }
     __syncthreads();
   }
@@ -237,7 +284,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
   }
   __syncthreads();
   long long tot;
-  const long long incl = block_inclusive_scan(part, scan_scratch, &tot);
+  const long long incl = block_inclusive_scan(part, scan_scratch[0], &tot);
   long long run = incl - part;
   for (int k = 0; k < per; ++k) {
     const int bin = nbins - 1 - (tid * per + k);

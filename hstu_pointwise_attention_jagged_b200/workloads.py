@@ -94,48 +94,52 @@ def make_custom(name, uih_len, num_targets, H, d, alpha, N, seed, cached_len=Non
                    cached_len, scale, bf16)
 
 
-def _finish(rng, name, uih, nt, H, d, alpha, N, cached_len, scale, bf16, meta=None):
+def _finish(rng, name, uih, nt, H, d, alpha, N, cached_len, scale, bf16, meta=None, values=True):
     B = len(uih)
     cl = np.zeros(B, np.int64) if cached_len is None else np.asarray(cached_len, np.int64)
     off = offsets_from_lengths(uih + nt)
     total = int(off[-1])
-    q, k, v = _draw(rng, total, H, d, (1.0 / math.sqrt(d)) if scale is None else scale, bf16)
+    if values:
+        q, k, v = _draw(rng, total, H, d, (1.0 / math.sqrt(d)) if scale is None else scale, bf16)
+    else:
+        q = k = v = np.zeros((0, H, d), np.float32)
     return Workload(name=name, B=B, H=H, d=d, alpha=float(alpha), N=float(N), uih_len=uih.astype(np.int32),
                     num_targets=nt.astype(np.int32), cached_len=cl.astype(np.int32), seq_offsets=off,
                     q=q, k=k, v=v, bf16=bf16, meta=meta or {})
 
 
 # The five named workloads: (description, builder).
-def _tiny(seed=0):
+def _tiny(seed=0, values=True):
     rng = np.random.default_rng(seed)
     uih = rng.integers(16, 64, size=4, endpoint=True).astype(np.int64)
-    return _finish(rng, "tiny", uih, np.full(4, 4, np.int64), 2, 32, 1 / math.sqrt(32), 68, None, None, False)
+    return _finish(rng, "tiny", uih, np.full(4, 4, np.int64), 2, 32, 1 / math.sqrt(32), 68, None, None, False,
+                   values=values)
 
 
-def _dlrmv3(seed=1):
+def _dlrmv3(seed=1, values=True):
     rng = np.random.default_rng(seed)
     return _finish(rng, "dlrmv3", np.full(8, 2048, np.int64), np.full(8, 2048, np.int64), 4, 128,
-                   1 / math.sqrt(128), 4096, None, None, True)
+                   1 / math.sqrt(128), 4096, None, None, True, values=values)
 
 
-def _jagged(seed=2):
+def _jagged(seed=2, values=True):
     rng = np.random.default_rng(seed)
     u = rng.lognormal(mean=math.log(1024.0), sigma=1.0, size=64)
     uih = np.clip(np.rint(u), 32, 4096).astype(np.int64)
     return _finish(rng, "jagged", uih, np.full(64, 16, np.int64), 4, 128, 1 / math.sqrt(128), 4112, None, None,
-                   True)
+                   True, values=values)
 
 
-def _long(seed=3):
+def _long(seed=3, values=True):
     rng = np.random.default_rng(seed)
     return _finish(rng, "long_history", np.full(4, 8192, np.int64), np.full(4, 512, np.int64), 8, 64,
-                   1 / 8.0, 8704, None, None, True)
+                   1 / 8.0, 8704, None, None, True, values=values)
 
 
-def _streaming(seed=4):
+def _streaming(seed=4, values=True):
     rng = np.random.default_rng(seed)
     return _finish(rng, "streaming", np.full(16, 3300, np.int64), np.full(16, 2048, np.int64), 4, 128,
-                   1 / math.sqrt(128), 5348, np.full(16, 3000, np.int64), None, True)
+                   1 / math.sqrt(128), 5348, np.full(16, 3000, np.int64), None, True, values=values)
 
 
 CONFIGS = {
@@ -157,3 +161,11 @@ def make(name: str, seed=None) -> Workload:
     w = fn() if seed is None else fn(seed)
     w.meta["description"] = desc
     return w
+
+
+def structure(name: str, seed=None):
+    """The per-user lengths of a named workload without drawing its Q/K/V: (uih_len, num_targets,
+    cached_len, H, d, alpha, N), the same lengths that ``make(name, seed)`` draws."""
+    _, fn = CONFIGS[name]
+    w = fn(values=False) if seed is None else fn(seed, values=False)
+    return w.uih_len, w.num_targets, w.cached_len, w.H, w.d, w.alpha, w.N

@@ -228,6 +228,57 @@ hstu_status_t hstu_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                     void* out, void* stream);
 
 /*
+ * hstu_attn_bwd — backward pass of hstu_attn_fwd for training: the gradients of a scalar loss
+ * with respect to q, k and v, given its gradient dout with respect to out.  The pages print no
+ * backward pass; the infolabhq.com multi-stage page (scaling section) is about training such
+ * models, and the forward definition above fixes the gradients by the chain rule.  For every
+ * user, head and visible pair (i, j), with x = alpha <q_i, k_j>:
+ *
+ *     dv[j] += silu(x) * dout[i] / N
+ *     ds     = (<dout[i], v[j]> / N) * silu'(x) * alpha,   silu'(x) = sigma(x) (1 + x (1 - sigma(x)))
+ *     dq[i] += ds * k[j],      dk[j] += ds * q[i]
+ *
+ * Masked pairs contribute nothing.  Products accumulate in fp32 on the tensor cores; silu(x) and
+ * ds are rounded to bf16 before their matrix products, and the gradients to bf16 once.
+ *
+ *   q, k, v, dout   device, bf16 [total_tokens, H, d], 16-byte aligned (the forward's inputs and
+ *                   the loss gradient of its output).
+ *   seq_offsets, num_targets, B, H, d, total_tokens, max_seq_len, alpha, N: as in hstu_attn_fwd
+ *                   (full sequences; there is no cached form).
+ *   dq, dk, dv      device, bf16 [total_tokens, H, d], written; none may overlap an input or
+ *                   another gradient.  Rows of users skipped for inconsistent offsets are not
+ *                   written.
+ *   stream          cudaStream_t as void*.
+ * A stream-ordered plan buffer is taken from the library's pool and returned, as in
+ * hstu_attn_fwd.  Errors as in hstu_attn_fwd; inputs must be finite (as there).
+ */
+hstu_status_t hstu_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
+                            const int32_t* seq_offsets, const int32_t* num_targets,
+                            int32_t B, int32_t H, int32_t d,
+                            int32_t total_tokens, int32_t max_seq_len,
+                            float alpha, float N,
+                            void* dq, void* dk, void* dv, void* stream);
+
+/*
+ * hstu_attn_partition — splits one jagged batch across `parts` GPUs (host function, no GPU work).
+ * Users are independent: no row of one user reads another user's K/V (the mask of hstu_attn_fwd),
+ * so a batch shards by user with no exchange between GPUs.  Following the jagged layout of the
+ * TorchRec tutorial (voagi.com, section 2.1: concatenated values plus lengths), each GPU takes a
+ * contiguous run of users, users [user_start[p], user_start[p+1]) for GPU p, so that its rows are
+ * one contiguous block of q, k, v and out; its seq_offsets are the batch's, rebased to 0.
+ * The runs minimise the largest per-GPU cost, the cost of a user being its number of visible
+ * (query, key) pairs (the algorithmic work of its attention); trailing runs may be empty.
+ *   seq_offsets   HOST int32 [B+1];  num_targets, cached_len: HOST int32 [B] or NULL (all 0).
+ *   user_start    HOST int32 [parts+1], written.
+ * Returns HSTU_ERR_INVALID_ARGUMENT for B < 0, parts < 1 or NULL pointers, HSTU_ERR_BAD_OFFSETS for
+ * inconsistent lengths, else HSTU_OK.  The pages have no multi-GPU scheme for this step; this is
+ * the plain sharding that the layout allows.
+ */
+hstu_status_t hstu_attn_partition(const int32_t* seq_offsets, const int32_t* num_targets,
+                                  const int32_t* cached_len, int32_t B, int32_t parts,
+                                  int32_t* user_start);
+
+/*
  * hstu_attn_get_error — synchronises `stream`, returns the device error word of the current
  * device as a status (HSTU_OK if clean) and clears it.  The word is shared by all calls on
  * the device, so a nonzero status may come from any call completed since the last read.

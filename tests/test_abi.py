@@ -21,7 +21,8 @@ def test_header_declares_the_entry_points():
                                            "hstu_attn_plan_bytes",
                                            "hstu_attn_plan", "hstu_attn_fwd_planned", "hstu_attn_fwd_noalloc",
                                            "hstu_attn_get_error", "hstu_attn_status_string",
-                                           "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16"])
+                                           "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16",
+                                           "hstu_attn_bwd", "hstu_attn_partition"])
 
 
 def test_library_exports_every_declared_symbol(cuda_lib):
@@ -107,3 +108,26 @@ def test_zero_rows_need_no_pointers(cuda_lib):
     """With no query rows nothing is read or written: NULL token pointers are accepted."""
     assert _fwd(cuda_lib, q=None, k=None, v=None, out=None, total=0, B=3) == 0
     assert _fwd(cuda_lib, q=None, k=None, v=None, out=None, off=None, total=0, B=0) == 0
+
+
+def test_host_validation_bwd(cuda_lib):
+    """The backward entry rejects bad sizes, misalignment and overlapping gradients on the host."""
+    vp = ctypes.c_void_p
+    f = cuda_lib.hstu_attn_bwd
+    i32, f32 = ctypes.c_int32, ctypes.c_float
+    f.argtypes = [vp] * 6 + [i32] * 5 + [f32, f32] + [vp] * 4
+    mb = 1 << 20
+
+    def call(q=mb, k=2 * mb, v=3 * mb, do=4 * mb, dq=5 * mb, dk=6 * mb, dv=7 * mb, d=64, N=1.0, B=1, total=16):
+        return f(vp(q), vp(k), vp(v), vp(do), vp(4096), None, B, 2, d, total, 16, 1.0, N, vp(dq), vp(dk), vp(dv), None)
+
+    assert call(d=48) == 2
+    assert call(N=0.0) == 1
+    assert call(B=-1) == 1
+    assert call(do=None) == 1
+    assert call(dk=None) == 1
+    assert call(dv=4 * mb) == 1          # dv overlaps dout
+    assert call(dk=5 * mb) == 1          # dk overlaps dq
+    assert call(dq=mb + 64) == 1         # dq overlaps q
+    assert call(do=4 * mb + 8) == 2      # misaligned dout
+    assert call(q=None, k=None, v=None, do=None, dq=None, dk=None, dv=None, total=0) == 0

@@ -74,3 +74,22 @@ def test_reference_arm_rank0_only(monkeypatch):
     line = json.loads(buf.getvalue())
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["unit"] == "TFLOP/s"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_rank_workload_splits_one_batch():
+    """With two ranks the bench splits one batch of two replicas of the jagged workload into two
+    contiguous runs of users whose visible-pair costs differ by less than one user's cost."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from hstu_pointwise_attention_jagged_b200 import metrics
+    w0, n0 = bench.rank_workload("jagged", 2, 0)
+    w1, n1 = bench.rank_workload("jagged", 2, 1)
+    assert n0 == n1 == 128
+    assert w0.meta["users"][0] == 0 and w0.meta["users"][1] == w1.meta["users"][0] and w1.meta["users"][1] == 128
+    assert w0.B + w1.B == 128
+    c = [metrics.algorithmic_flops(w.seq_offsets, w.num_targets, w.H, w.d) for w in (w0, w1)]
+    largest = max(metrics.algorithmic_flops(w.seq_offsets[b:b + 2] - w.seq_offsets[b], w.num_targets[b:b + 1], w.H,
+                                            w.d) for w in (w0, w1) for b in range(w.B))
+    assert abs(c[0] - c[1]) <= largest
+    one, n = bench.rank_workload("dlrmv3", 1, 0)
+    assert n == 8 and one.B == 8

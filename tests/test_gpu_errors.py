@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_util import assert_parity, dev_bf16, dev_i32, to_f64
+from gpu_util import assert_parity, dev_bf16, dev_i32, row_users, to_f64
 from hstu_pointwise_attention_jagged_b200 import binding, workloads
 
 pytestmark = pytest.mark.gpu
@@ -36,7 +36,7 @@ def test_bad_targets_skip_user_and_report():
     s = w.seq_offsets
     assert np.all(o[s[1]:s[2]] == 5.0)
     keep = np.r_[s[0]:s[1], s[2]:s[3]]
-    assert_parity(o[keep], ref[keep], what="valid users")
+    assert_parity(o[keep], ref[keep], what="valid users", users=row_users(w)[keep])
 
 
 def test_user_longer_than_max_seq_len_is_skipped():
@@ -47,7 +47,7 @@ def test_user_longer_than_max_seq_len_is_skipped():
     assert binding.hstu_attn_get_error() == 4
     assert torch.all(out[:300] == 5.0)
     ref = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, None, w.alpha, w.N)
-    assert_parity(to_f64(out[300:]), ref[300:], what="short user")
+    assert_parity(to_f64(out[300:]), ref[300:], what="short user", users=row_users(w)[300:])
 
 
 def test_cached_prefix_into_candidates_is_rejected():
@@ -88,10 +88,34 @@ def test_bounded_wait_times_out_and_reports():
                                 dev_i32(w.num_targets), w.alpha, w.N, w.max_seq_len)
     assert binding.hstu_attn_get_error() == 0
     ref = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N)
-    assert_parity(to_f64(out), ref, what="after a timed-out self-check")
+    assert_parity(to_f64(out), ref, what="after a timed-out self-check", users=row_users(w))
 
 
 def test_selfcheck_rejects_out_of_range_limits():
     for bad in (0, 2_000_000_000):
         with pytest.raises(binding.HstuError):
             binding.hstu_attn_selfcheck_wait_timeout(bad)
+
+
+def test_corrupt_lengths_near_int_max_write_nothing_outside_out():
+    """Two corrupt users whose lengths are about 2^31 rows, then a well-formed user.  The plan
+    kernel takes lengths in 64 bits and caps a corrupt user's rows, so no query-row start wraps
+    negative: the call reports HSTU_ERR_BAD_OFFSETS, no work item points outside `out`, and the
+    guard rows on both sides of `out` keep their sentinel."""
+    off = np.array([0, 2147483000, -5, 2147483000, 0, 100], np.int32)
+    nt = np.zeros(5, np.int32)
+    H, d, total = 2, 64, 100
+    plan = binding.hstu_attn_plan(dev_i32(off), dev_i32(nt), None, H, total, total, 100)
+    _, q_start, items = binding.plan_contents(plan, 5)
+    assert binding.hstu_attn_get_error() == 4
+    assert all(int(s) == -1 or 0 <= int(s) < total for s in q_start)
+    for it in items:
+        assert 0 <= int(q_start[int(it[0])]) < total
+    rng = np.random.default_rng(35)
+    q = dev_bf16(workloads.round_bf16(rng.standard_normal((total, H, d), dtype=np.float32) / 8))
+    pad = 256
+    big = torch.full((total + 2 * pad, H, d), 7.0, dtype=torch.bfloat16, device="cuda")
+    binding.hstu_attn_fwd(q, q, q, dev_i32(off), dev_i32(nt), 0.125, 100.0, 100, out=big[pad:pad + total])
+    torch.cuda.synchronize()
+    assert binding.hstu_attn_get_error() == 4
+    assert torch.all(big[:pad] == 7.0) and torch.all(big[pad + total:] == 7.0)

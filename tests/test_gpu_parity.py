@@ -16,7 +16,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_util import (assert_parity, dev_bf16, dev_i32, query_row_index, rel_l2, run_cached, run_fwd,
+from gpu_util import (assert_parity, dev_bf16, dev_i32, query_row_index, rel_l2, row_users, run_cached, run_fwd,
                       sample_rows, to_f64)
 from hstu_pointwise_attention_jagged_b200 import binding, workloads
 
@@ -26,7 +26,7 @@ pytestmark = pytest.mark.gpu
 def _full_compare(w, what):
     got = to_f64(run_fwd(w))
     ref = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N)
-    return assert_parity(got, ref, what=what)
+    return assert_parity(got, ref, what=what, users=row_users(w))
 
 
 def test_tiny_config():
@@ -59,7 +59,7 @@ def test_plain_causal_without_num_targets():
     w = workloads.make_custom("causal", [200, 1, 77, 400], [0, 0, 0, 0], 2, 128, 1 / math.sqrt(128), 400.0, seed=7)
     got = to_f64(run_fwd(w, num_targets=None))
     ref = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, None, w.alpha, w.N)
-    assert_parity(got, ref, what="num_targets=NULL")
+    assert_parity(got, ref, what="num_targets=NULL", users=row_users(w))
 
 
 def test_stress_large_scores():
@@ -69,7 +69,7 @@ def test_stress_large_scores():
         w = workloads.make_custom("stress", [190, 31, 260], [20, 5, 1], 2, d, 1.0, 64.0, seed=9, scale=1.0)
         got = to_f64(run_fwd(w))
         ref = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N)
-        assert_parity(got, ref, max_abs=1e-2 * np.abs(ref).max(), what="stress d=%d" % d)
+        assert_parity(got, ref, max_abs=1e-2 * np.abs(ref).max(), what="stress d=%d" % d, users=row_users(w))
 
 
 def test_many_small_users():
@@ -94,7 +94,7 @@ def test_single_long_user():
     rows = query_row_index(w, users, local)
     got = to_f64(got_all[torch.from_numpy(rows).cuda()])
     ref = oracle.rows(w.q, w.k, w.v, w.seq_offsets, w.num_targets, None, w.alpha, w.N, users, local)
-    assert_parity(got, ref, what="single 32K-token user")
+    assert_parity(got, ref, what="single 32K-token user", users=users)
     assert torch.isfinite(got_all.float()).all()
 
 
@@ -107,7 +107,7 @@ def test_full_size_sampled(name):
     rows = query_row_index(w, users, local)
     got = to_f64(got_all[torch.from_numpy(rows).cuda()])
     ref = oracle.rows(w.q, w.k, w.v, w.seq_offsets, w.num_targets, None, w.alpha, w.N, users, local)
-    assert_parity(got, ref, what=name)
+    assert_parity(got, ref, what=name, users=users)
     assert torch.isfinite(got_all.float()).all()
 
 
@@ -121,9 +121,10 @@ def test_streaming_config():
     users, local = sample_rows(w, cached=True)
     rows = query_row_index(w, users, local, cached=True)
     ref = oracle.rows(w.q[sel], w.k, w.v, w.seq_offsets, w.num_targets, w.cached_len, w.alpha, w.N, users, local)
-    assert_parity(to_f64(got_c[torch.from_numpy(rows).cuda()]), ref, what="streaming vs oracle")
+    assert_parity(to_f64(got_c[torch.from_numpy(rows).cuda()]), ref, what="streaming vs oracle", users=users)
     full = run_fwd(w, k=k, v=v)
-    assert_parity(to_f64(got_c), to_f64(full[torch.from_numpy(sel).cuda()]), what="streaming vs full recompute")
+    assert_parity(to_f64(got_c), to_f64(full[torch.from_numpy(sel).cuda()]), what="streaming vs full recompute",
+                  users=row_users(w, cached=True))
 
 
 def test_cached_small_full_compare():
@@ -133,7 +134,7 @@ def test_cached_small_full_compare():
     got = to_f64(run_cached(w))
     sel = w.new_rows()
     ref = oracle.fwd_cached(w.q[sel], w.k, w.v, w.seq_offsets, w.num_targets, w.cached_len, w.alpha, w.N)
-    assert_parity(got, ref, what="cached small")
+    assert_parity(got, ref, what="cached small", users=row_users(w, cached=True))
 
 
 def test_cached_zero_prefix_equals_full_bitwise():
@@ -172,7 +173,7 @@ def test_no_writes_outside_user_rows():
     run_fwd(w, out=big[pad:pad + w.total])
     assert torch.all(big[:pad] == 7.0) and torch.all(big[pad + w.total:] == 7.0)
     ref = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N)
-    assert_parity(to_f64(big[pad:pad + w.total]), ref, what="guard")
+    assert_parity(to_f64(big[pad:pad + w.total]), ref, what="guard", users=row_users(w))
 
 
 def test_empty_batches_are_noops():

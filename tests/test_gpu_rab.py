@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_util import assert_parity, dev_bf16, dev_i32, query_row_index, sample_rows, to_f64
+from gpu_util import assert_parity, dev_bf16, dev_i32, query_row_index, row_users, sample_rows, to_f64
 from hstu_pointwise_attention_jagged_b200 import binding, workloads
 
 pytestmark = pytest.mark.gpu
@@ -34,7 +34,7 @@ def test_rab_ragged(d):
     rab = _table(H, 300, seed=d)
     got = to_f64(_run(w, rab))
     ref = oracle.fwd_rab(w.q, w.k, w.v, w.seq_offsets, w.num_targets, rab, w.alpha, w.N)
-    assert_parity(got, ref, what="rab ragged d=%d" % d)
+    assert_parity(got, ref, what="rab ragged d=%d" % d, users=row_users(w))
 
 
 def test_rab_zero_table_is_plain_attention():
@@ -55,9 +55,10 @@ def test_rab_cached_matches_oracle_and_full():
     got = _run(w, rab, q=dev_bf16(w.q[sel]), cached_len=w.cached_len)
     ref = oracle.fwd_rab(w.q[sel], w.k, w.v, w.seq_offsets, w.num_targets, rab, w.alpha, w.N,
                          cached_len=w.cached_len)
-    assert_parity(to_f64(got), ref, what="rab cached vs oracle")
+    assert_parity(to_f64(got), ref, what="rab cached vs oracle", users=row_users(w, cached=True))
     full = _run(w, rab)
-    assert_parity(to_f64(got), to_f64(full[torch.from_numpy(sel).cuda()]), what="rab cached vs full")
+    assert_parity(to_f64(got), to_f64(full[torch.from_numpy(sel).cuda()]), what="rab cached vs full",
+                  users=row_users(w, cached=True))
 
 
 def test_rab_full_size_sampled():
@@ -69,5 +70,5 @@ def test_rab_full_size_sampled():
     rows = query_row_index(w, users, local)
     got = to_f64(got_all[torch.from_numpy(rows).cuda()])
     ref = oracle.rows_rab(w.q, w.k, w.v, w.seq_offsets, w.num_targets, None, rab, w.alpha, w.N, users, local)
-    assert_parity(got, ref, what="rab dlrmv3")
+    assert_parity(got, ref, what="rab dlrmv3", users=users)
     assert binding.hstu_attn_get_error() == 0
