@@ -581,6 +581,224 @@ def run_proj(args, ranks):
     return line
 
 
+def run_bwd(args, ranks):
+    """Backward pass (hstu_attn_bwd: plan, dK/dV kernel, dQ kernel) over this rank's share of the
+    workload, with a seeded N(0,1) output gradient.  Algorithmic flops are the five mask-exact
+    matmuls of the chain rule (S, dP, dV, dK, dQ: 10 d flops per visible pair and head); the two
+    the dQ kernel recomputes are not counted."""
+    import torch
+    from hstu_pointwise_attention_jagged_b200 import binding, metrics, workloads
+
+    dev = torch.device("cuda", ranks.local_rank)
+    torch.cuda.set_device(dev)
+    binding.load_library()
+    w, global_users = rank_workload(args.workload, ranks.world, ranks.rank)
+    if w.cached_len.any():
+        raise SystemExit("--variant bwd: the backward pass takes full sequences (no cached prefix)")
+    flops = metrics.algorithmic_flops(w.seq_offsets, w.num_targets, w.H, w.d) * 10 // 4
+
+    def to_bf16(x):
+        return torch.from_numpy(workloads.bf16_bits(x).view(np.int16)).view(torch.bfloat16)
+
+    do = workloads.round_bf16(np.random.default_rng(rank_seed(6, ranks.rank)).standard_normal(
+        w.q.shape, dtype=np.float32))
+    host = [to_bf16(x).pin_memory() for x in (w.q, w.k, w.v, do)]
+    q, k, v, dout = (x.to(dev) for x in host)
+    off = torch.from_numpy(w.seq_offsets.astype(np.int32)).to(dev)
+    nt = torch.from_numpy(w.num_targets.astype(np.int32)).to(dev)
+    grads = [torch.empty_like(q) for _ in range(3)]
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        binding.hstu_attn_bwd(q, k, v, dout, off, nt, w.alpha, w.N, w.max_seq_len, dq=grads[0], dk=grads[1],
+                              dv=grads[2], stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if binding.hstu_attn_get_error() != 0:
+        raise RuntimeError("warm-up reported an error")
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    ranks.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        ranks.barrier()
+    if binding.hstu_attn_get_error() != 0:
+        raise RuntimeError("timed steps reported an error")
+    ms = ranks.max(sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)), dev) / K
+    job_flops = ranks.sum(flops, dev)
+    value = job_flops / (ms * 1e-3) / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    peak, peak_src = measured_peak()
+
+    # End to end: q, k, v, dout and the offsets from pinned host memory, the three gradients back.
+    off_h = torch.from_numpy(w.seq_offsets.astype(np.int32)).pin_memory()
+    nt_h = torch.from_numpy(w.num_targets.astype(np.int32)).pin_memory()
+    grads_h = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(3)]
+    h2d = sum(x.numel() * x.element_size() for x in host + [off_h, nt_h])
+    d2h = sum(g.numel() * g.element_size() for g in grads_h)
+    E = max(4, min(args.steps, 50))
+
+    def e2e_step():
+        for dst, src in zip((q, k, v, dout, off, nt), host + [off_h, nt_h]):
+            dst.copy_(src, non_blocking=True)
+        step()
+        for gh, g in zip(grads_h, grads):
+            gh.copy_(g, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ranks.max(e0.elapsed_time(e1), dev) / E
+    line = {
+        "metric": "jagged SiLU-attention backward TFLOP/s (dQ, dK, dV)",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ranks.world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1)/sqrt(d) bf16 inputs, N(0,1) output gradient)",
+        "config": dict(workload_config(w, ranks.world, global_users), variant="backward pass"),
+        "e2e": {"value": round(job_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 3 * (K + E),
+        "roofline": {"bound": "tensor", "kernel": "hstu_bwd_kernel<%d, dK/dV> + <%d, dQ> (+ plan)" % (w.d, w.d),
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None, "peak_source": peak_src,
+                     "flops_per_step": int(flops)},
+        "clocks": sampler.summary(),
+    }
+    return line
+
+
+LAYERS = 3  # stacked HSTU layers for --variant layer
+
+
+def run_layer(args, ranks):
+    """A stack of HSTU layers (projection GEMM, attention with the [U | A | U*A] epilogue, projection
+    GEMM; one work plan for all layers) through hstu_layers_fwd, on this rank's share of the
+    workload with D = H d.  `value` counts the review's per-layer FLOP formula,
+    2 * layers * sum_users (L*L*D/2 + 4*L*D^2 + 3*L*D^2) with L each user's length (DLRMv3 review,
+    section "model selection"); the mask-exact count (projections plus visible pairs) is reported
+    beside it."""
+    import torch
+    from hstu_pointwise_attention_jagged_b200 import binding, metrics, workloads
+
+    dev = torch.device("cuda", ranks.local_rank)
+    torch.cuda.set_device(dev)
+    binding.load_library()
+    w, global_users = rank_workload(args.workload, ranks.world, ranks.rank)
+    if w.cached_len.any():
+        raise SystemExit("--variant layer: layers take full sequences (no cached prefix)")
+    H, d, D, L = w.H, w.d, w.H * w.d, w.total
+    lens = w.seq_len
+    page_flops = int(2 * LAYERS * sum(int(l) * int(l) * D // 2 + 7 * int(l) * D * D for l in lens))
+    exact_flops = LAYERS * (2 * L * D * 7 * D + metrics.algorithmic_flops(w.seq_offsets, w.num_targets, H, d))
+    rng = np.random.default_rng(rank_seed(12, ranks.rank))
+
+    def bf16(a):
+        return torch.from_numpy(workloads.bf16_bits(workloads.round_bf16(a.astype(np.float32))).view(np.int16)).view(
+            torch.bfloat16)
+
+    x_h = bf16(rng.standard_normal((L, D))).pin_memory()
+    w1 = [bf16(rng.standard_normal((4 * D, D)) / np.sqrt(D)).to(dev) for _ in range(LAYERS)]
+    w2 = [bf16(rng.standard_normal((D, 3 * D)) / np.sqrt(3 * D)).to(dev) for _ in range(LAYERS)]
+    x = x_h.to(dev)
+    off_h = torch.from_numpy(w.seq_offsets.astype(np.int32)).pin_memory()
+    nt_h = torch.from_numpy(w.num_targets.astype(np.int32)).pin_memory()
+    off, nt = off_h.to(dev), nt_h.to(dev)
+    ws = torch.empty((binding.hstu_layer_workspace_bytes(H, d, L, LAYERS),), dtype=torch.uint8, device=dev)
+    y = torch.empty_like(x)
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        binding.hstu_layers_fwd(x, w1, w2, off, nt, H, d, w.alpha, w.N, w.max_seq_len, workspace=ws, y=y,
+                                stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if binding.hstu_attn_get_error() != 0:
+        raise RuntimeError("warm-up reported an error")
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    ranks.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        ranks.barrier()
+    if binding.hstu_attn_get_error() != 0:
+        raise RuntimeError("timed steps reported an error")
+    ms = ranks.max(sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)), dev) / K
+    job_page = ranks.sum(page_flops, dev)
+    job_exact = ranks.sum(exact_flops, dev)
+    peak, peak_src = measured_peak()
+
+    # End to end: the input activations and offsets from pinned host memory, the output back.
+    y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    E = max(4, min(args.steps, 50))
+
+    def e2e_step():
+        x.copy_(x_h, non_blocking=True)
+        off.copy_(off_h, non_blocking=True)
+        nt.copy_(nt_h, non_blocking=True)
+        step()
+        y_h.copy_(y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ranks.max(e0.elapsed_time(e1), dev) / E
+    h2d = sum(t.numel() * t.element_size() for t in (x_h, off_h, nt_h))
+    return {
+        "metric": "HSTU layer stack TFLOP/s by the review's formula 2*layers*(L^2 D/2 + 7 L D^2)",
+        "value": round(job_page / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": ranks.world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, bf16)",
+        "config": dict(workload_config(w, ranks.world, global_users), layers=LAYERS, model_dim=D,
+                       variant="HSTU layer stack: [U|V|Q|K] = X W1^T, attention, Y = [U|A|U*A] W2^T"),
+        "exact_tflops": round(job_exact / (ms * 1e-3) / 1e12, 2),
+        "page_gflop_per_step": round(job_page / 1e9, 3), "exact_gflop_per_step": round(job_exact / 1e9, 3),
+        "e2e": {"value": round(job_page / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(y_h.numel() * y_h.element_size())},
+        "gpu_launches": (1 + 3 * LAYERS) * (K + E),
+        "roofline": {"bound": "tensor", "kernel": "layer stack (gemm_bf16_kernel x2 + hstu_fwd_kernel per layer)",
+                     "achieved": round(exact_flops / (ms * 1e-3) / 1e12, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(exact_flops / (ms * 1e-3) / 1e12 / peak, 4), "traffic": None,
+                     "peak_source": peak_src, "flops_per_step": int(exact_flops)},
+        "clocks": sampler.summary(),
+    }
+
+
 def run_reference(args, world):
     """The fp64 oracle on the host cores, rank 0 only: each step a bounded row sample, sized so that
     warm-up plus K steps stay near a minute of CPU work."""
@@ -630,9 +848,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOAD_SEEDS), default=WORKLOAD,
                     help="batch to time (default: the DLRMv3-shaped benchmark batch)")
-    ap.add_argument("--variant", choices=["plain", "rab", "proj"], default="plain",
-                    help="rab: the relative-attention-bias variant (a %d-entry table per head); proj: the layer's "
-                         "projection GEMMs" % RAB_LEN)
+    ap.add_argument("--variant", choices=["plain", "rab", "proj", "bwd", "layer"], default="plain",
+                    help="layer: a stack of %d HSTU layers; bwd: the backward pass; rab: the relative-attention-bias variant (a %d-entry table per "
+                         "head); proj: the layer's "
+                         "projection GEMMs" % (LAYERS, RAB_LEN))
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of this kernel, if current")
     args = ap.parse_args(argv)
@@ -648,7 +867,8 @@ def main(argv=None):
         return 0
     ranks = Ranks(backend="nccl")
     try:
-        line = run_proj(args, ranks) if args.variant == "proj" else run_ours(args, ranks)
+        run = {"proj": run_proj, "bwd": run_bwd, "layer": run_layer}.get(args.variant, run_ours)
+        line = run(args, ranks)
     finally:
         ranks.close()
     if ranks.rank == 0:

@@ -38,6 +38,9 @@ EXPORTS = (
     "hstu_attn_gemm_bf16",
     "hstu_attn_bwd",
     "hstu_attn_partition",
+    "hstu_layer_workspace_bytes",
+    "hstu_layer_fwd",
+    "hstu_layers_fwd",
 )
 
 
@@ -82,10 +85,15 @@ def load_library():
     lib.hstu_attn_gemm_bf16.argtypes = [vp, vp, vp, i32, i32, i32, vp]
     lib.hstu_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp, vp]
     lib.hstu_attn_partition.argtypes = [vp, vp, vp, i32, i32, vp]
+    lib.hstu_layer_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    lib.hstu_layer_workspace_bytes.restype = i64
+    lib.hstu_layer_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, f32, vp, vp, i64, vp, vp]
+    lib.hstu_layers_fwd.argtypes = [i32, vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, vp, i32, i32, i32, i32, i32,
+                                    f32, f32, vp, i64, vp, vp]
     lib.hstu_attn_status_string.restype = ctypes.c_char_p
     for name in ("hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_fwd_rab", "hstu_attn_plan", "hstu_attn_fwd_planned",
                  "hstu_attn_get_error", "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16", "hstu_attn_bwd",
-                 "hstu_attn_partition"):
+                 "hstu_attn_partition", "hstu_layer_fwd", "hstu_layers_fwd"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -385,3 +393,73 @@ def shard_of(seq_offsets, user_start, part):
     u0, u1 = int(user_start[part]), int(user_start[part + 1])
     r0, r1 = int(off[u0]), int(off[u1])
     return u0, u1, r0, r1, (off[u0:u1 + 1] - r0).astype(np.int32)
+
+
+def hstu_layer_workspace_bytes(H, d, total, num_layers=1):
+    return int(load_library().hstu_layer_workspace_bytes(int(H), int(d), int(total), int(num_layers)))
+
+
+def _check_act(name, t, D):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 2 or \
+            t.shape[1] != D or not t.is_contiguous():
+        raise TypeError("%s must be a contiguous bf16 CUDA tensor [rows, %d]" % (name, D))
+
+
+def hstu_layer_fwd(x, w_uvqk, w_out, seq_offsets, num_targets, H, d, alpha, N, plan, workspace=None, y=None,
+                   stream=None):
+    """One HSTU layer (projection, attention, projection) over a plan from hstu_attn_plan; returns y
+    (bf16 [total, H*d]). See include/hstu_attn.h."""
+    lib = load_library()
+    D = H * d
+    _check_act("x", x, D)
+    total = x.shape[0]
+    _check_act("w_uvqk", w_uvqk, D)
+    _check_act("w_out", w_out, 3 * D)
+    if w_uvqk.shape[0] != 4 * D or w_out.shape[0] != D:
+        raise ValueError("w_uvqk must be [4D, D] and w_out [D, 3D]")
+    B = seq_offsets.numel() - 1
+    _check_index("seq_offsets", seq_offsets, B + 1, x.device, optional=False)
+    _check_index("num_targets", num_targets, B, x.device)
+    nbytes = hstu_layer_workspace_bytes(H, d, total, 1)
+    if workspace is None:
+        workspace = torch.empty((nbytes,), dtype=torch.uint8, device=x.device)
+    y = torch.empty_like(x) if y is None else y
+    _check_act("y", y, D)
+    with torch.cuda.device(x.device):
+        st = lib.hstu_layer_fwd(_ptr(x), _ptr(w_uvqk), _ptr(w_out), _ptr(seq_offsets), _ptr(num_targets), B, H, d,
+                                total, float(alpha), float(N), _ptr(plan), _ptr(workspace), workspace.numel(),
+                                _ptr(y), _stream_ptr(stream, x.device))
+    _raise_if(st, "hstu_layer_fwd")
+    return y
+
+
+def hstu_layers_fwd(x, w_uvqk_list, w_out_list, seq_offsets, num_targets, H, d, alpha, N, max_seq_len,
+                    workspace=None, y=None, stream=None):
+    """A stack of HSTU layers over one work plan; returns the last layer's output. See
+    include/hstu_attn.h."""
+    lib = load_library()
+    D = H * d
+    L = len(w_uvqk_list)
+    if L < 1 or len(w_out_list) != L:
+        raise ValueError("need one w_uvqk and one w_out per layer")
+    _check_act("x", x, D)
+    for w1, w2 in zip(w_uvqk_list, w_out_list):
+        _check_act("w_uvqk", w1, D)
+        _check_act("w_out", w2, 3 * D)
+    total = x.shape[0]
+    B = seq_offsets.numel() - 1
+    _check_index("seq_offsets", seq_offsets, B + 1, x.device, optional=False)
+    _check_index("num_targets", num_targets, B, x.device)
+    nbytes = hstu_layer_workspace_bytes(H, d, total, L)
+    if workspace is None:
+        workspace = torch.empty((nbytes,), dtype=torch.uint8, device=x.device)
+    y = torch.empty_like(x) if y is None else y
+    _check_act("y", y, D)
+    w1p = (ctypes.c_void_p * L)(*[w.data_ptr() for w in w_uvqk_list])
+    w2p = (ctypes.c_void_p * L)(*[w.data_ptr() for w in w_out_list])
+    with torch.cuda.device(x.device):
+        st = lib.hstu_layers_fwd(L, _ptr(x), w1p, w2p, _ptr(seq_offsets), _ptr(num_targets), B, H, d, total,
+                                 int(max_seq_len), float(alpha), float(N), _ptr(workspace), workspace.numel(), _ptr(y),
+                                 _stream_ptr(stream, x.device))
+    _raise_if(st, "hstu_layers_fwd")
+    return y

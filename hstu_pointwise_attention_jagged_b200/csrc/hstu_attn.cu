@@ -104,11 +104,12 @@ bool encoder() {
   return g_encode != nullptr;
 }
 
-// 2-D bf16 tensor map over a jagged [rows, H*d] matrix; box = (box_x columns, 128 rows).
+// 2-D bf16 tensor map over a jagged [rows, H*d] matrix whose rows are `ld` elements apart (ld = 0:
+// packed, H*d); box = (box_x columns, 128 rows).
 bool encode_rows(CUtensorMap* map, const void* base, int64_t rows, int64_t row_elems, uint32_t box_x,
-                 CUtensorMapSwizzle swz) {
+                 CUtensorMapSwizzle swz, int64_t ld = 0) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_elems), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_elems) * 2u};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld > 0 ? ld : row_elems) * 2u};
   cuuint32_t box[2] = {box_x, static_cast<cuuint32_t>(kTileRows)};
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
@@ -246,19 +247,30 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   return cudaLaunchKernelEx(&cfg, hstu_fwd_kernel<D, kRab>, tq, tk, tv, p);
 }
 
+// Row strides and the layer epilogue's extra streams for a call whose tensors are column blocks
+// of wider matrices (the HSTU layer); every stride 0 means packed [rows, H, d].
+struct StridedIO {
+  int64_t q_ld = 0, kv_ld = 0, out_ld = 0;
+  const void* gate = nullptr;
+  int64_t gate_ld = 0;
+  void* gate_copy = nullptr;
+  void* gate_prod = nullptr;
+};
+
 // The attention kernel over a plan built for the same offsets.  Arguments already checked.
 hstu_status_t launch_attention(DeviceState* st, const void* q, const void* k, const void* v,
                                const int32_t* seq_offsets, const int32_t* num_targets, const int32_t* cached_len,
                                int32_t B, int32_t H, int32_t d, int32_t total_kv, int32_t total_q, float alpha,
                                float N, void* plan, void* out, cudaStream_t stream, const float* rab = nullptr,
-                               int32_t rab_len = 0) {
+                               int32_t rab_len = 0, const StridedIO& io = StridedIO()) {
   if (!encoder()) return HSTU_ERR_CUDA;
   const int64_t row_elems = static_cast<int64_t>(H) * d;
   CUtensorMap tq, tk, tv;
   const uint32_t box_x = d >= 64 ? 64u : 32u;
   const CUtensorMapSwizzle swz = d >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  if (!encode_rows(&tq, q, total_q, row_elems, box_x, swz) || !encode_rows(&tk, k, total_kv, row_elems, box_x, swz) ||
-      !encode_rows(&tv, v, total_kv, row_elems, box_x, swz))
+  if (!encode_rows(&tq, q, total_q, row_elems, box_x, swz, io.q_ld) ||
+      !encode_rows(&tk, k, total_kv, row_elems, box_x, swz, io.kv_ld) ||
+      !encode_rows(&tv, v, total_kv, row_elems, box_x, swz, io.kv_ld))
     return HSTU_ERR_CUDA;
   const Plan w = carve(plan, B);
   FwdParams p;
@@ -271,6 +283,11 @@ hstu_status_t launch_attention(DeviceState* st, const void* q, const void* k, co
   p.work_counter = w.counter;
   p.done_counter = w.done;
   p.out = static_cast<__nv_bfloat16*>(out);
+  p.out_ld = io.out_ld > 0 ? io.out_ld : row_elems;
+  p.gate = static_cast<const __nv_bfloat16*>(io.gate);
+  p.gate_ld = io.gate_ld;
+  p.gate_copy = static_cast<__nv_bfloat16*>(io.gate_copy);
+  p.gate_prod = static_cast<__nv_bfloat16*>(io.gate_prod);
   p.rab = rab;
   p.rab_len = rab_len;
   p.H = H;
@@ -290,6 +307,75 @@ hstu_status_t launch_attention(DeviceState* st, const void* q, const void* k, co
     else e = launch_fwd<32, false>(tq, tk, tv, p, grid, stream);
   }
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// C = A W^T on the projection GEMM kernel.  Arguments already checked.
+hstu_status_t launch_gemm(DeviceState* st, const void* a, const void* w, void* c, int32_t M, int32_t N, int32_t K,
+                          cudaStream_t stream) {
+  if (!encoder()) return HSTU_ERR_CUDA;
+  CUtensorMap ta, tw;
+  if (!encode_matrix(&ta, a, M, K, kGemmBM) || !encode_matrix(&tw, w, N, K, kGemmBN)) return HSTU_ERR_CUDA;
+  GemmParams p;
+  p.c = static_cast<__nv_bfloat16*>(c);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.tiles_m = (M + kGemmBM - 1) / kGemmBM;
+  p.tiles_n = (N + kGemmBN - 1) / kGemmBN;
+  p.err = st->err_word;
+  const int64_t ntiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+  if (ntiles > INT_MAX) return HSTU_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(ntiles < st->num_sms ? ntiles : st->num_sms);
+  gemm_bf16_kernel<<<grid, kGemmThreads, GemmCfg::kSmemBytes, stream>>>(ta, tw, p);
+  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// One HSTU layer over a plan built for its offsets (full sequences):
+//   UVQK = X W_uvqk^T                     [total, 4D]: blocks U, V, Q, K of D = H d columns
+//   A = attention(Q, K, V)                read in place from UVQK; written into CAT[:, D:2D]
+//   CAT[:, 0:D] = U, CAT[:, 2D:3D] = U*A  by the attention epilogue
+//   Y = CAT W_out^T                       [total, D]
+// workspace holds UVQK then CAT.  Arguments already checked.
+hstu_status_t run_layer(DeviceState* st, const void* x, const void* w_uvqk, const void* w_out,
+                        const int32_t* seq_offsets, const int32_t* num_targets, int32_t B, int32_t H, int32_t d,
+                        int32_t total, float alpha, float N, void* plan, void* workspace, void* y,
+                        cudaStream_t stream) {
+  const int64_t D = static_cast<int64_t>(H) * d;
+  auto* uvqk = static_cast<__nv_bfloat16*>(workspace);
+  auto* cat = uvqk + static_cast<size_t>(total) * 4 * D;
+  hstu_status_t s = launch_gemm(st, x, w_uvqk, uvqk, total, static_cast<int32_t>(4 * D), static_cast<int32_t>(D),
+                                stream);
+  if (s != HSTU_OK) return s;
+  StridedIO io;
+  io.q_ld = io.kv_ld = 4 * D;
+  io.out_ld = 3 * D;
+  io.gate = uvqk;
+  io.gate_ld = 4 * D;
+  io.gate_copy = cat;
+  io.gate_prod = cat + 2 * D;
+  s = launch_attention(st, uvqk + 2 * D, uvqk + 3 * D, uvqk + D, seq_offsets, num_targets, nullptr, B, H, d, total,
+                       total, alpha, N, plan, cat + D, stream, nullptr, 0, io);
+  if (s != HSTU_OK) return s;
+  return launch_gemm(st, cat, w_out, y, total, static_cast<int32_t>(D), static_cast<int32_t>(3 * D), stream);
+}
+
+// Checks shared by the layer entry points.
+hstu_status_t check_layer(const void* x, const void* y, const void* workspace, const int32_t* seq_offsets,
+                          int32_t B, int32_t H, int32_t d, int32_t total, float alpha, float N) {
+  hstu_status_t s = check_sizes(B, H, total, total);
+  if (s != HSTU_OK) return s;
+  if (!std::isfinite(alpha) || !std::isfinite(N) || !(N > 0.0f)) return HSTU_ERR_INVALID_ARGUMENT;
+  if (d != 32 && d != 64 && d != 128) return HSTU_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(H) * d * 4 > INT_MAX / 2) return HSTU_ERR_UNSUPPORTED;
+  if (total == 0 || B == 0) return HSTU_OK;
+  if (!x || !y || !workspace || !seq_offsets) return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(workspace)) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+int64_t layer_workspace_bytes(int32_t H, int32_t d, int32_t total, int32_t layers) {
+  const int64_t D = static_cast<int64_t>(H) * d;
+  return static_cast<int64_t>(total) * D * 2 * (7 + (layers > 1 ? 1 : 0));
 }
 
 // Plan into a stream-ordered buffer from the library's pool, attention, return the buffer.
@@ -590,24 +676,8 @@ hstu_status_t hstu_attn_gemm_bf16(const void* a, const void* w, void* c, int32_t
                cc = static_cast<size_t>(M) * N * 2;
   if (hstu::overlaps(c, cc, a, ca) || hstu::overlaps(c, cc, w, cw)) return HSTU_ERR_INVALID_ARGUMENT;
   hstu::DeviceState* st = hstu::device_state();
-  if (!st || !hstu::encoder()) return HSTU_ERR_CUDA;
-  CUtensorMap ta, tw;
-  if (!hstu::encode_matrix(&ta, a, M, K, hstu::kGemmBM) || !hstu::encode_matrix(&tw, w, N, K, hstu::kGemmBN))
-    return HSTU_ERR_CUDA;
-  hstu::GemmParams p;
-  p.c = static_cast<__nv_bfloat16*>(c);
-  p.M = M;
-  p.N = N;
-  p.K = K;
-  p.tiles_m = (M + hstu::kGemmBM - 1) / hstu::kGemmBM;
-  p.tiles_n = (N + hstu::kGemmBN - 1) / hstu::kGemmBN;
-  p.err = st->err_word;
-  const int64_t ntiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-  if (ntiles > INT_MAX) return HSTU_ERR_UNSUPPORTED;
-  const int grid = static_cast<int>(ntiles < st->num_sms ? ntiles : st->num_sms);
-  hstu::gemm_bf16_kernel<<<grid, hstu::kGemmThreads, hstu::GemmCfg::kSmemBytes,
-                           static_cast<cudaStream_t>(stream_ptr)>>>(ta, tw, p);
-  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  if (!st) return HSTU_ERR_CUDA;
+  return hstu::launch_gemm(st, a, w, c, M, N, K, static_cast<cudaStream_t>(stream_ptr));
 }
 
 hstu_status_t hstu_attn_partition(const int32_t* seq_offsets, const int32_t* num_targets,
@@ -660,6 +730,71 @@ hstu_status_t hstu_attn_partition(const int32_t* seq_offsets, const int32_t* num
   }
   for (int32_t k = part + 1; k <= parts; ++k) user_start[k] = B;
   return HSTU_OK;
+}
+
+int64_t hstu_layer_workspace_bytes(int32_t H, int32_t d, int32_t total, int32_t num_layers) {
+  if (H < 1 || d < 1 || total < 0 || num_layers < 1) return 0;
+  return hstu::layer_workspace_bytes(H, d, total, num_layers);
+}
+
+hstu_status_t hstu_layer_fwd(const void* x, const void* w_uvqk, const void* w_out, const int32_t* seq_offsets,
+                             const int32_t* num_targets, int32_t B, int32_t H, int32_t d, int32_t total,
+                             float alpha, float N, void* plan, void* workspace, int64_t workspace_bytes, void* y,
+                             void* stream_ptr) {
+  hstu_status_t s = hstu::check_layer(x, y, workspace, seq_offsets, B, H, d, total, alpha, N);
+  if (s != HSTU_OK || total == 0 || B == 0) return s;
+  if (!w_uvqk || !w_out || !plan) return HSTU_ERR_INVALID_ARGUMENT;
+  if (!hstu::aligned16(w_uvqk) || !hstu::aligned16(w_out) || !hstu::aligned16(plan)) return HSTU_ERR_UNSUPPORTED;
+  if (workspace_bytes < hstu::layer_workspace_bytes(H, d, total, 1)) return HSTU_ERR_INVALID_ARGUMENT;
+  const size_t act = static_cast<size_t>(total) * H * d * 2;
+  if (hstu::overlaps(y, act, workspace, static_cast<size_t>(workspace_bytes)) ||
+      hstu::overlaps(x, act, workspace, static_cast<size_t>(workspace_bytes)))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  hstu::DeviceState* st = hstu::device_state();
+  if (!st) return HSTU_ERR_CUDA;
+  return hstu::run_layer(st, x, w_uvqk, w_out, seq_offsets, num_targets, B, H, d, total, alpha, N, plan, workspace,
+                         y, static_cast<cudaStream_t>(stream_ptr));
+}
+
+hstu_status_t hstu_layers_fwd(int32_t num_layers, const void* x, const void* const* w_uvqk,
+                              const void* const* w_out, const int32_t* seq_offsets, const int32_t* num_targets,
+                              int32_t B, int32_t H, int32_t d, int32_t total, int32_t max_seq_len, float alpha,
+                              float N, void* workspace, int64_t workspace_bytes, void* y, void* stream_ptr) {
+  if (num_layers < 1 || !w_uvqk || !w_out || max_seq_len < 0) return HSTU_ERR_INVALID_ARGUMENT;
+  hstu_status_t s = hstu::check_layer(x, y, workspace, seq_offsets, B, H, d, total, alpha, N);
+  if (s != HSTU_OK || total == 0 || B == 0) return s;
+  for (int32_t l = 0; l < num_layers; ++l) {
+    if (!w_uvqk[l] || !w_out[l]) return HSTU_ERR_INVALID_ARGUMENT;
+    if (!hstu::aligned16(w_uvqk[l]) || !hstu::aligned16(w_out[l])) return HSTU_ERR_UNSUPPORTED;
+  }
+  if (workspace_bytes < hstu::layer_workspace_bytes(H, d, total, num_layers)) return HSTU_ERR_INVALID_ARGUMENT;
+  const size_t act = static_cast<size_t>(total) * H * d * 2;
+  if (hstu::overlaps(y, act, workspace, static_cast<size_t>(workspace_bytes)) ||
+      hstu::overlaps(x, act, workspace, static_cast<size_t>(workspace_bytes)))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  hstu::DeviceState* st = hstu::device_state();
+  if (!st) return HSTU_ERR_CUDA;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  // One plan for every layer: the jagged structure does not change between layers.
+  void* plan = nullptr;
+  if (cudaMallocFromPoolAsync(&plan, static_cast<size_t>(hstu::plan_bytes(B, H, total)), st->pool, stream) !=
+      cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (hstu::launch_plan(seq_offsets, num_targets, nullptr, B, H, total, total, max_seq_len, hstu::carve(plan, B),
+                        st->err_word, stream) != cudaSuccess)
+    s = HSTU_ERR_CUDA;
+  // Layer l reads its input (x, then the hidden buffer after UVQK and CAT) and writes its output
+  // (y for the last layer); a layer's input is dead once its first projection has run, so the
+  // hidden buffer can be read and rewritten by the same layer.
+  auto* hidden = static_cast<uint8_t*>(workspace) + static_cast<size_t>(total) * H * d * 2 * 7;
+  for (int32_t l = 0; l < num_layers && s == HSTU_OK; ++l) {
+    const void* in = l == 0 ? x : hidden;
+    void* out = l == num_layers - 1 ? y : hidden;
+    s = hstu::run_layer(st, in, w_uvqk[l], w_out[l], seq_offsets, num_targets, B, H, d, total, alpha, N, plan,
+                        workspace, out, stream);
+  }
+  if (cudaFreeAsync(plan, stream) != cudaSuccess && s == HSTU_OK) s = HSTU_ERR_CUDA;
+  return s;
 }
 
 hstu_status_t hstu_attn_selfcheck_wait_timeout(uint64_t limit_ns, void* stream_ptr) {

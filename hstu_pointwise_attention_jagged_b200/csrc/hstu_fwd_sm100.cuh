@@ -74,6 +74,13 @@ struct FwdParams {
   int32_t* work_counter;
   int32_t* done_counter;
   __nv_bfloat16* out;
+  int64_t out_ld;              // elements between consecutive rows of out (H*D when packed)
+  // Layer epilogue (all null outside a layer): with gate = U, also writes U to gate_copy and
+  // U * A (A rounded to bf16 first) to gate_prod, rows strided like out; U rows are gate_ld apart.
+  const __nv_bfloat16* gate;
+  int64_t gate_ld;
+  __nv_bfloat16* gate_copy;
+  __nv_bfloat16* gate_prod;
   const float* rab;            // relative-bias variant: [H, rab_len] table; unused otherwise
   int32_t rab_len;
   int32_t H;
@@ -147,6 +154,13 @@ __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Elementwise product of two bf16 pairs, each product formed in fp32 and rounded to bf16 once.
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+  const float a0 = __uint_as_float(a << 16), a1 = __uint_as_float(a & 0xffff0000u);
+  const float b0 = __uint_as_float(b << 16), b1 = __uint_as_float(b & 0xffff0000u);
+  return pack_bf16x2(a0 * b0, a1 * b1);
 }
 
 // SiLU + mask + bf16 pack of 32 score columns [32*chunk, 32*chunk+32) of this thread's row,
@@ -531,22 +545,41 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       if (!ok) break;
       o_full_par ^= 1u;
       ptx::tc_fence_after();
-      __nv_bfloat16* dst = p.out + ((size_t)(w.q_row0 + lo + row) * p.H + w.h) * D;
+      const size_t orow = (size_t)(w.q_row0 + lo + row);
+      __nv_bfloat16* dst = p.out + orow * p.out_ld + (size_t)w.h * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ro[32];
         ptx::tmem_ld32(taddr_o + c * 32, ro);
         ptx::tmem_ld_wait(ro);
         if (row < nr) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+          uint4 a4[4];
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 0]) * inv_n, __uint_as_float(ro[q4 * 8 + 1]) * inv_n);
-            v.y = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 2]) * inv_n, __uint_as_float(ro[q4 * 8 + 3]) * inv_n);
-            v.z = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 4]) * inv_n, __uint_as_float(ro[q4 * 8 + 5]) * inv_n);
-            v.w = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 6]) * inv_n, __uint_as_float(ro[q4 * 8 + 7]) * inv_n);
-            d4[q4] = v;
+            a4[q4].x = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 0]) * inv_n, __uint_as_float(ro[q4 * 8 + 1]) * inv_n);
+            a4[q4].y = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 2]) * inv_n, __uint_as_float(ro[q4 * 8 + 3]) * inv_n);
+            a4[q4].z = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 4]) * inv_n, __uint_as_float(ro[q4 * 8 + 5]) * inv_n);
+            a4[q4].w = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 6]) * inv_n, __uint_as_float(ro[q4 * 8 + 7]) * inv_n);
+            reinterpret_cast<uint4*>(dst + c * 32)[q4] = a4[q4];
+          }
+          if (p.gate != nullptr) {
+            // Layer epilogue: the gate row U, a copy of it and U * A, beside A in the next
+            // projection's input.
+            const size_t col = (size_t)w.h * D + c * 32;
+            const uint4* u4 = reinterpret_cast<const uint4*>(p.gate + orow * p.gate_ld + col);
+            uint4* cp4 = reinterpret_cast<uint4*>(p.gate_copy + orow * p.out_ld + col);
+            uint4* pr4 = reinterpret_cast<uint4*>(p.gate_prod + orow * p.out_ld + col);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const uint4 u = u4[q4];
+              cp4[q4] = u;
+              uint4 pr;
+              pr.x = mul_bf16x2(u.x, a4[q4].x);
+              pr.y = mul_bf16x2(u.y, a4[q4].y);
+              pr.z = mul_bf16x2(u.z, a4[q4].z);
+              pr.w = mul_bf16x2(u.w, a4[q4].w);
+              pr4[q4] = pr;
+            }
           }
         }
       }

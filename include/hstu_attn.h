@@ -305,6 +305,56 @@ hstu_status_t hstu_attn_gemm_bf16(const void* a, const void* w, void* c, int32_t
                              void* stream);
 
 /*
+ * HSTU layer: the attention step between the two dense projections whose flops the DLRMv3 review
+ * counts per layer as 4*L*D^2 and 3*L*D^2 (section "model selection", FLOP-formula paragraph:
+ * 2 * layers * (L*L*D/2 + 4*L*D^2 + 3*L*D^2)), with layers stacked as the infolabhq.com multi-stage
+ * page describes (section "Target-Aware Multi-Head Attention").  The pages give only the flop
+ * terms; the layer built here is the plainest composition with exactly those terms (D = H * d):
+ *
+ *     UVQK = X W_uvqk^T        X [total, D], W_uvqk [4D, D]  -> [total, 4D] = [U | V | Q | K]
+ *     A    = hstu_attn_fwd(Q, K, V)                         (each a [total, H, d] view of UVQK)
+ *     Y    = [U | A | U*A] W_out^T                           W_out [D, 3D] -> Y [total, D]
+ *
+ * U*A is elementwise.  No normalisation, activation or residual is added: the pages name none.
+ * All tensors are bf16, row-major, on the device; products accumulate in fp32 and every stored
+ * tensor (UVQK, A, U*A, Y) is rounded to bf16 once.  The attention reads Q, K, V in place and its
+ * epilogue writes U, A and U*A straight into the second projection's input, so the layer is
+ * three kernels over one work plan.
+ *
+ * hstu_layer_workspace_bytes — device bytes of the workspace for num_layers stacked layers
+ *   (UVQK, the [U | A | U*A] buffer and, for more than one layer, the hidden activations):
+ *   total * D * 2 * (7 + (num_layers > 1)); 0 for invalid sizes.
+ *
+ * hstu_layer_fwd — one layer over a plan built by hstu_attn_plan(seq_offsets, num_targets, NULL,
+ *   B, H, total, total, ...) (the plan may be reused by every layer of the batch).
+ *   x, y          device bf16 [total, D]; y must not overlap the workspace; x may equal y.
+ *   w_uvqk, w_out device bf16 [4D, D] and [D, 3D] (out-features x in-features), 16-byte aligned.
+ *   seq_offsets, num_targets, B, H, d, total, alpha, N: as in hstu_attn_fwd.
+ *   workspace     device, >= hstu_layer_workspace_bytes(H, d, total, 1) bytes, 16-byte aligned.
+ *
+ * hstu_layers_fwd — num_layers layers, layer l using w_uvqk[l] and w_out[l] (HOST arrays of
+ *   device pointers); builds one plan (from the library's pool, like hstu_attn_fwd) and reuses it
+ *   for every layer.  x is the first layer's input, y the last layer's output.
+ *
+ * Errors as in hstu_attn_fwd and hstu_attn_gemm_bf16 (HSTU_ERR_INVALID_ARGUMENT for a short
+ * workspace or one that overlaps x or y); asynchronous on `stream`.
+ */
+int64_t hstu_layer_workspace_bytes(int32_t H, int32_t d, int32_t total, int32_t num_layers);
+
+hstu_status_t hstu_layer_fwd(const void* x, const void* w_uvqk, const void* w_out,
+                             const int32_t* seq_offsets, const int32_t* num_targets,
+                             int32_t B, int32_t H, int32_t d, int32_t total,
+                             float alpha, float N, void* plan,
+                             void* workspace, int64_t workspace_bytes, void* y, void* stream);
+
+hstu_status_t hstu_layers_fwd(int32_t num_layers, const void* x,
+                              const void* const* w_uvqk, const void* const* w_out,
+                              const int32_t* seq_offsets, const int32_t* num_targets,
+                              int32_t B, int32_t H, int32_t d, int32_t total, int32_t max_seq_len,
+                              float alpha, float N,
+                              void* workspace, int64_t workspace_bytes, void* y, void* stream);
+
+/*
  * hstu_attn_selfcheck_wait_timeout — exercises the failure-detection path on `stream`: one
  * thread of a one-warp kernel waits, through the same bounded mbarrier wait every role of the
  * attention kernel uses, on a barrier that nothing arrives on.  After limit_ns nanoseconds

@@ -245,3 +245,48 @@ def linear(a, w):
     """C = A · Wᵀ in fp64 (A [M, K], W [N, K]): the dense projections of the HSTU layer whose flops
     the DLRMv3 review counts as 4·L·D² and 3·L·D² per layer.  A matrix product is the definition."""
     return np.asarray(a, np.float64) @ np.asarray(w, np.float64).T
+
+
+def round_bf16(a):
+    """Rounds to the nearest bf16 value, ties to even (the storage format of every tensor the library
+    passes between steps), returned as float64.  Written from the format: keep the top 16 bits of the
+    float32 pattern, rounding the dropped 16 bits to nearest with ties to the even kept pattern."""
+    f = np.ascontiguousarray(np.asarray(a, np.float64).astype(np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    keep = u >> np.uint64(16)
+    rest = u & np.uint64(0xFFFF)
+    up = (rest > 0x8000) | ((rest == 0x8000) & ((keep & np.uint64(1)) == 1))
+    keep = keep + up.astype(np.uint64)
+    return (keep << np.uint64(16)).astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def layer(x, w_uvqk, w_out, seq_offsets, num_targets, H, d, alpha, N):
+    """One HSTU layer as the library composes it, from oracle.linear and oracle.fwd only (fp64, with
+    every tensor the library stores between its steps rounded to bf16):
+
+        UVQK = X W_uvqk^T   -> blocks U, V, Q, K of D = H d columns
+        A    = attention(Q, K, V)
+        Y    = [U | A | U*A] W_out^T
+
+    The DLRMv3 review (section "model selection", FLOP-formula paragraph) gives the layer's flops as
+    4 L D^2 + L^2 D / 2 + 3 L D^2; the blocks above are the plainest reading with those terms.
+    Returns Y [total, D] in fp64 (not rounded)."""
+    x = np.asarray(x, np.float64)
+    total, D = x.shape
+    uvqk = round_bf16(linear(x, w_uvqk))
+    u, v, q, k = (uvqk[:, i * D:(i + 1) * D] for i in range(4))
+    a = fwd(q.reshape(total, H, d), k.reshape(total, H, d), v.reshape(total, H, d), seq_offsets, num_targets,
+            alpha, N).reshape(total, D)
+    a = round_bf16(a)
+    cat = np.concatenate([u, a, round_bf16(u * a)], axis=1)
+    return linear(cat, w_out)
+
+
+def layers(x, w_uvqk_list, w_out_list, seq_offsets, num_targets, H, d, alpha, N):
+    """A stack of layers; the hidden activations between layers are stored as bf16."""
+    y = np.asarray(x, np.float64)
+    for i, (w1, w2) in enumerate(zip(w_uvqk_list, w_out_list)):
+        if i > 0:
+            y = round_bf16(y)
+        y = layer(y, w1, w2, seq_offsets, num_targets, H, d, alpha, N)
+    return y

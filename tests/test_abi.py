@@ -13,7 +13,7 @@ HEADER = os.path.join(ROOT, "include", "hstu_attn.h")
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(hstu_attn_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(hstu_(?:attn|layer|layers)_\w+)\s*\(", text)))
 
 
 def test_header_declares_the_entry_points():
@@ -22,7 +22,8 @@ def test_header_declares_the_entry_points():
                                            "hstu_attn_plan", "hstu_attn_fwd_planned", "hstu_attn_fwd_noalloc",
                                            "hstu_attn_get_error", "hstu_attn_status_string",
                                            "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16",
-                                           "hstu_attn_bwd", "hstu_attn_partition"])
+                                           "hstu_attn_bwd", "hstu_attn_partition", "hstu_layer_workspace_bytes",
+                                           "hstu_layer_fwd", "hstu_layers_fwd"])
 
 
 def test_library_exports_every_declared_symbol(cuda_lib):
