@@ -41,6 +41,7 @@ EXPORTS = (
     "hstu_layer_workspace_bytes",
     "hstu_layer_fwd",
     "hstu_layers_fwd",
+    "hstu_attn_selfcheck_fwd_timeout",
 )
 
 
@@ -85,6 +86,8 @@ def load_library():
     lib.hstu_attn_gemm_bf16.argtypes = [vp, vp, vp, i32, i32, i32, vp]
     lib.hstu_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp, vp]
     lib.hstu_attn_partition.argtypes = [vp, vp, vp, i32, i32, vp]
+    lib.hstu_attn_selfcheck_fwd_timeout.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp,
+                                                    ctypes.c_uint64, vp]
     lib.hstu_layer_workspace_bytes.argtypes = [i32, i32, i32, i32]
     lib.hstu_layer_workspace_bytes.restype = i64
     lib.hstu_layer_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, f32, vp, vp, i64, vp, vp]
@@ -93,7 +96,8 @@ def load_library():
     lib.hstu_attn_status_string.restype = ctypes.c_char_p
     for name in ("hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_fwd_rab", "hstu_attn_plan", "hstu_attn_fwd_planned",
                  "hstu_attn_get_error", "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16", "hstu_attn_bwd",
-                 "hstu_attn_partition", "hstu_layer_fwd", "hstu_layers_fwd"):
+                 "hstu_attn_partition", "hstu_layer_fwd", "hstu_layers_fwd",
+                 "hstu_attn_selfcheck_fwd_timeout"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -463,3 +467,19 @@ def hstu_layers_fwd(x, w_uvqk_list, w_out_list, seq_offsets, num_targets, H, d, 
                                  _stream_ptr(stream, x.device))
     _raise_if(st, "hstu_layers_fwd")
     return y
+
+
+def hstu_attn_selfcheck_fwd_timeout(q, k, v, seq_offsets, num_targets, alpha, N, max_seq_len, limit_ns, out=None,
+                                    stream=None):
+    """hstu_attn_fwd with every attention-kernel wait limited to limit_ns (test hook of the abort path)."""
+    lib = load_library()
+    _check_tokens("q", q)
+    total, H, d = q.shape
+    B = seq_offsets.numel() - 1
+    out = torch.empty_like(q) if out is None else out
+    with torch.cuda.device(q.device):
+        st = lib.hstu_attn_selfcheck_fwd_timeout(_ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(num_targets), B,
+                                                 H, d, total, int(max_seq_len), float(alpha), float(N), _ptr(out),
+                                                 int(limit_ns), _stream_ptr(stream, q.device))
+    _raise_if(st, "hstu_attn_selfcheck_fwd_timeout")
+    return out

@@ -255,6 +255,7 @@ struct StridedIO {
   int64_t gate_ld = 0;
   void* gate_copy = nullptr;
   void* gate_prod = nullptr;
+  uint64_t wait_limit_ns = kWaitLimitNs;
 };
 
 // The attention kernel over a plan built for the same offsets.  Arguments already checked.
@@ -294,6 +295,7 @@ hstu_status_t launch_attention(DeviceState* st, const void* q, const void* k, co
   p.half_alpha = 0.5f * alpha;
   p.inv_n = 1.0f / N;
   p.err = st->err_word;
+  p.wait_limit_ns = io.wait_limit_ns;
   const int64_t cap = capacity(B, H, total_q);
   const int grid = static_cast<int>(cap < st->num_sms ? cap : st->num_sms);
   cudaError_t e;
@@ -803,6 +805,34 @@ hstu_status_t hstu_attn_selfcheck_wait_timeout(uint64_t limit_ns, void* stream_p
   if (!st) return HSTU_ERR_CUDA;
   hstu::wait_timeout_selfcheck_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_ptr)>>>(st->err_word, limit_ns);
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status_t hstu_attn_selfcheck_fwd_timeout(const void* q, const void* k, const void* v,
+                                              const int32_t* seq_offsets, const int32_t* num_targets, int32_t B,
+                                              int32_t H, int32_t d, int32_t total_tokens, int32_t max_seq_len,
+                                              float alpha, float N, void* out, uint64_t limit_ns, void* stream_ptr) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return HSTU_ERR_INVALID_ARGUMENT;
+  hstu_status_t s = hstu::check_sizes(B, H, total_tokens, total_tokens);
+  if (s == HSTU_OK && max_seq_len < 0) s = HSTU_ERR_INVALID_ARGUMENT;
+  if (s == HSTU_OK) s = hstu::check_tokens(q, k, v, seq_offsets, H, d, total_tokens, total_tokens, alpha, N, out);
+  if (s != HSTU_OK || B == 0 || total_tokens == 0) return s;
+  hstu::DeviceState* st = hstu::device_state();
+  if (!st) return HSTU_ERR_CUDA;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  void* plan = nullptr;
+  if (cudaMallocFromPoolAsync(&plan, static_cast<size_t>(hstu::plan_bytes(B, H, total_tokens)), st->pool, stream) !=
+      cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (hstu::launch_plan(seq_offsets, num_targets, nullptr, B, H, total_tokens, total_tokens, max_seq_len,
+                        hstu::carve(plan, B), st->err_word, stream) != cudaSuccess)
+    s = HSTU_ERR_CUDA;
+  hstu::StridedIO io;
+  io.wait_limit_ns = limit_ns;
+  if (s == HSTU_OK)
+    s = hstu::launch_attention(st, q, k, v, seq_offsets, num_targets, nullptr, B, H, d, total_tokens, total_tokens,
+                               alpha, N, plan, out, stream, nullptr, 0, io);
+  if (cudaFreeAsync(plan, stream) != cudaSuccess && s == HSTU_OK) s = HSTU_ERR_CUDA;
+  return s;
 }
 
 const char* hstu_attn_status_string(hstu_status_t s) {

@@ -87,6 +87,7 @@ struct FwdParams {
   float half_alpha;
   float inv_n;
   unsigned* err;
+  uint64_t wait_limit_ns;      // limit of every pipeline wait (kWaitLimitNs; a self-check lowers it)
 };
 
 template <int kStages>
@@ -285,7 +286,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const int rows = (w.L - c) - pair * kPairRows;
           w.nrows = rows < kPairRows ? rows : kPairRows;
         }
-        if (!wait_bounded(bar(ctl->sched_empty[slot]), sched_empty_par[slot], abort_flag, p.err)) break;
+        if (!wait_bounded(bar(ctl->sched_empty[slot]), sched_empty_par[slot], abort_flag, p.err, p.wait_limit_ns)) break;
         sched_empty_par[slot] ^= 1u;
         volatile int32_t* s = ctl->slot[slot];
         s[0] = w.valid; s[1] = w.h; s[2] = w.kv_start; s[3] = w.q_row0;
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
         const TileRange un = key_tiles(w.pos0, w.pos0 + w.nrows, w.U);
         const int n_u = tile_count(un);
-        if (!wait_bounded(bar(ctl->q_empty), q_empty_par, abort_flag, p.err)) break;
+        if (!wait_bounded(bar(ctl->q_empty), q_empty_par, abort_flag, p.err, p.wait_limit_ns)) break;
         q_empty_par ^= 1u;
         ptx::mbar_arrive_expect_tx(bar(ctl->q_full), 2 * Cfg::kTileBytes);
         for (int hh = 0; hh < 2; ++hh)
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         for (int i = 0; i < n_u && ok; ++i) {
           const int row = w.kv_start + tile_at(un, i) * kTileRows;
           for (int kv = 0; kv < 2; ++kv) {
-            if (!wait_bounded(bar(ctl->kv_empty[stage]), kv_phase ^ 1u, abort_flag, p.err)) {
+            if (!wait_bounded(bar(ctl->kv_empty[stage]), kv_phase ^ 1u, abort_flag, p.err, p.wait_limit_ns)) {
               ok = false;
               break;
             }
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const uint32_t lead = (lane == 0) ? 1u : 0u;
     // Waits are taken by every lane and the outcome is made warp-uniform.
     auto wait_all = [&](uint32_t b, uint32_t par) {
-      return __all_sync(0xffffffffu, wait_bounded(b, par, abort_flag, p.err));
+      return __all_sync(0xffffffffu, wait_bounded(b, par, abort_flag, p.err, p.wait_limit_ns));
     };
     // Descriptor templates: the descriptor of address a + off is template(a) + (off >> 4).
     const uint64_t dq0 = ptx::smem_desc(sQ, 16, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
@@ -471,7 +472,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     uint32_t s_full_par = 0u, o_full_par = 0u;
     bool ok = true;
     while (ok) {
-      ok = wait_bounded(bar(ctl->sched_full[slot]), sched_full_par[slot], abort_flag, p.err);
+      ok = wait_bounded(bar(ctl->sched_full[slot]), sched_full_par[slot], abort_flag, p.err, p.wait_limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       sched_full_par[slot] ^= 1u;
@@ -493,7 +494,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       const int rab_max = kRab ? p.rab_len - 1 : 0;
       for (int k = 0; k < n; ++k) {
         const int j0 = tile_at(r, k) * kTileRows;
-        ok = wait_bounded(bar(ctl->s_full[hh]), s_full_par, abort_flag, p.err);
+        ok = wait_bounded(bar(ctl->s_full[hh]), s_full_par, abort_flag, p.err, p.wait_limit_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         s_full_par ^= 1u;
@@ -540,7 +541,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       }
       if (!ok) break;
       // Epilogue: O_h * (1/N) -> bf16 -> out rows that exist.
-      ok = wait_bounded(bar(ctl->o_full[hh]), o_full_par, abort_flag, p.err);
+      ok = wait_bounded(bar(ctl->o_full[hh]), o_full_par, abort_flag, p.err, p.wait_limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       o_full_par ^= 1u;

@@ -366,6 +366,24 @@ hstu_status_t hstu_layers_fwd(int32_t num_layers, const void* x,
  */
 hstu_status_t hstu_attn_selfcheck_wait_timeout(uint64_t limit_ns, void* stream);
 
+/*
+ * hstu_attn_selfcheck_fwd_timeout — exercises the attention kernel's own abort path: the same work
+ * as hstu_attn_fwd, but every pipeline wait of the attention kernel gives up after limit_ns
+ * nanoseconds (1 .. 1e9) instead of the normal 4 s.  A wait that runs out sets the timeout bit of
+ * the device error word and raises the CTA's abort flag; every role then leaves its loop, waits
+ * (each wait at most 0.2 s) for the copies and MMAs it issued, TMEM is freed and the kernel
+ * returns, so the next hstu_attn_get_error reports HSTU_ERR_TIMEOUT and the context stays usable.
+ * `out` is left partly written.  Arguments and errors as in hstu_attn_fwd, plus
+ * HSTU_ERR_INVALID_ARGUMENT for a limit outside the range.  The pages have no counterpart: this is
+ * a test hook of the library's own failure handling.
+ */
+hstu_status_t hstu_attn_selfcheck_fwd_timeout(const void* q, const void* k, const void* v,
+                                              const int32_t* seq_offsets, const int32_t* num_targets,
+                                              int32_t B, int32_t H, int32_t d,
+                                              int32_t total_tokens, int32_t max_seq_len,
+                                              float alpha, float N, void* out,
+                                              uint64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,7 +23,7 @@ def test_header_declares_the_entry_points():
                                            "hstu_attn_get_error", "hstu_attn_status_string",
                                            "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16",
                                            "hstu_attn_bwd", "hstu_attn_partition", "hstu_layer_workspace_bytes",
-                                           "hstu_layer_fwd", "hstu_layers_fwd"])
+                                           "hstu_layer_fwd", "hstu_layers_fwd", "hstu_attn_selfcheck_fwd_timeout"])
 
 
 def test_library_exports_every_declared_symbol(cuda_lib):

@@ -119,3 +119,22 @@ def test_corrupt_lengths_near_int_max_write_nothing_outside_out():
     torch.cuda.synchronize()
     assert binding.hstu_attn_get_error() == 4
     assert torch.all(big[:pad] == 7.0) and torch.all(big[pad + total:] == 7.0)
+
+
+def test_attention_kernel_abort_path_then_recovers():
+    """The attention kernel itself with every pipeline wait limited to 1 µs: the waits that are not
+    met at once run out, the CTAs raise their abort flag, drain the copies and MMAs they issued,
+    free TMEM and return.  The device reports HSTU_ERR_TIMEOUT once, and a normal call on the same
+    context afterwards matches the oracle."""
+    w = workloads.make_custom("abort", [600, 300, 40], [100, 20, 2], 2, 128, 1 / math.sqrt(128), 700.0, seed=36)
+    q, k, v = dev_bf16(w.q), dev_bf16(w.k), dev_bf16(w.v)
+    off, nt = dev_i32(w.seq_offsets), dev_i32(w.num_targets)
+    assert binding.hstu_attn_get_error() == 0
+    for _ in range(2):
+        binding.hstu_attn_selfcheck_fwd_timeout(q, k, v, off, nt, w.alpha, w.N, w.max_seq_len, 1000)
+        assert binding.hstu_attn_get_error() == 5  # HSTU_ERR_TIMEOUT
+        assert binding.hstu_attn_get_error() == 0
+    out = binding.hstu_attn_fwd(q, k, v, off, nt, w.alpha, w.N, w.max_seq_len)
+    assert binding.hstu_attn_get_error() == 0
+    ref = oracle.fwd(w.q, w.k, w.v, w.seq_offsets, w.num_targets, w.alpha, w.N)
+    assert_parity(to_f64(out), ref, what="after an aborted attention kernel", users=row_users(w))
