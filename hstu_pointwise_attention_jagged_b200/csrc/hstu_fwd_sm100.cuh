@@ -121,13 +121,13 @@ __device__ __forceinline__ Work read_slot(const volatile int32_t* s) {
 }
 
 // Slow path of wait_bounded: spins until the phase completes, the CTA aborts, or the time limit.
+// Each try_wait may itself suspend the thread for a while, so the flag and the clock are checked
+// after every attempt.
 __device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag,
                                                unsigned* err, uint64_t limit_ns) {
   const uint64_t t0 = ptx::globaltimer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (ptx::mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (ptx::globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
