@@ -1,23 +1,35 @@
 // hstu_fwd_sm100.cuh — fused forward kernel of jagged target-aware HSTU pointwise attention for
 // sm_100a:  out = Mask(SiLU(alpha * Q K^T)) V / N   (DLRMv3 review, section "model selection").
 //
-// One persistent CTA per SM pulls work items (user b, head h, 256 query rows) from a cost-
-// ordered list through an atomic counter.  Per item the two 128-row halves share every K/V tile.
+// One persistent CTA per SM pulls work items (user b, head h, up to 256 query rows) from a cost-
+// ordered list through an atomic counter.  Each item is worked as one or two 128-row sub-items
+// (query tiles); every role walks the same global sequence of score tiles g = 0, 1, 2, ... over
+// the CTA's sub-items and their visible key tiles.
 //
-//   warp 8      producer: fetches the next item, TMA-loads Q (both halves) and the item's key
-//               tiles K_t, V_t into a ring of shared-memory stages (128B/64B swizzle).
-//   warp 9      MMA issuer: the warp runs converged and lane 0 issues every tcgen05 instruction.
-//               S_h = Q_h K_t^T into TMEM (SS form), then, once the SiLU warps have written P_h,
-//               O_h += P_h V_t with P_h read from TMEM (TS form).  Issue order per key tile:
-//               PV_0(prev) S_0(t) PV_1(prev) S_1(t), so the tensor core has the other half's work
-//               while one half's SiLU runs.
-//   warps 0-3   SiLU warpgroup of half 0, warps 4-7 of half 1: TMEM -> registers, p =
-//               mask ? silu(alpha*s) : 0 with silu(x) = h + h*tanh(h), h = x/2 (one MUFU op per
-//               score), packed to bf16 and written back over S in TMEM; after the item's last
-//               tile, the epilogue: O * (1/N) -> bf16 -> row-predicated global stores.
+//   warp 8       producer: fetches the next item, TMA-loads each sub-item's Q into one of two
+//                buffers and the K and V tiles into a ring of shared-memory slots, in the order
+//                the tensor core consumes them: K_0 K_1 K_2 V_0 K_3 V_1 K_4 ... (V_{g-3}, K_g).
+//   warp 9       MMA issuer (lane 0 issues every tcgen05 instruction).  Group g is
+//                O += P_{g-3} V_{g-3}  (TS form, P read from TMEM), then S_g = Q K_g^T into score
+//                buffer g mod 3 (SS form), then one commit.  Three score buffers give the SiLU of
+//                tile g two whole groups of tensor-core work to hide behind before P_g is needed.
+//   warps 0-3,   SiLU warpgroups; warpgroup g mod 2 takes tile g: TMEM -> registers, p = mask ?
+//   warps 4-7    silu(alpha*s) : 0 with silu(x) = h + h*tanh(h), h = x/2 (one MUFU op per score),
+//                packed to bf16 and written back over S_g in TMEM.
+//   warps 10-13  epilogue: after a sub-item's last P.V, O * (1/N) -> bf16 -> row-predicated
+//                global stores.  O is released as soon as it is in registers, so the next
+//                sub-item's first P.V waits only for the TMEM reads.
 //
-// TMEM (512 columns x 128 lanes of fp32): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
-// O_1 [256+D, 256+2D).  P_h (bf16 pairs) overwrites the first 64 columns of S_h.
+// TMEM (512 columns x 128 lanes of fp32): O [0, D), score buffer b at [128 + 128 b, 256 + 128 b)
+// for b = 0, 1, 2.  P_g (bf16 pairs) overwrites the first 64 columns of its score buffer; the
+// next S MMA into that buffer is issued after the P.V that reads it, and tcgen05 MMAs from one
+// thread execute in order.
+//
+// Each group has one ready barrier: the producer's copies for it (Q on a sub-item's first tile,
+// V_{g-3}, K_g) complete their bytes on it and the four SiLU warps that wrote P_{g-3} arrive on it,
+// so the MMA warp makes one wait per group.  A ring slot is reused once the group that consumed
+// its previous tile has completed; the score commit of group G covers every MMA issued before it,
+// so the producer waits on that commit and no separate release commit is needed.
 //
 // hstu_fwd_kernel<D, true> is the relative-attention-bias variant: each visible pair's p also gets
 // a per-head table entry for its query-key distance (the table is read through the read-only
@@ -37,6 +49,9 @@
 
 namespace hstu {
 
+constexpr int kSCommits = 6;      // score-commit barriers: tile g's S commit arrives on s_full[g mod 6]
+constexpr int kGroupBars = 8;     // group-ready barriers: group g waits on g_ready[g mod 8]
+
 template <int D>
 struct FwdCfg {
   static_assert(D == 32 || D == 64 || D == 128, "head size");
@@ -47,20 +62,30 @@ struct FwdCfg {
   static constexpr int kTileBytes = kBlocks * kBlockBytes;  // 128 rows x D bf16
   static constexpr uint32_t kSwizzle = (kRowBytes == 128) ? 2u : 4u;  // UMMA layout code
   static constexpr int kKStepsPerBlock = kBlockElems / 16;
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kQBufs = 2;
+  // K/V ring slots: as many as fit beside the two Q buffers in 227 KB.
+  static constexpr int kStages = (D == 128) ? 5 : 10;
+  static constexpr int kSBufs = 3;
+  // The producer reuses a ring slot after waiting on the score commit of the group that consumed
+  // the slot's previous tile.  That commit rotates over kSCommits barriers, so the wait is
+  // unambiguous only while group G + kSCommits cannot have completed yet, i.e. while its K tile
+  // (load 2 (G + kSCommits) - 2) is not yet loaded: at worst (G = 0, load kStages) that needs
+  // kStages <= 2 kSCommits - 2.
+  static_assert(kStages <= 2 * kSCommits - 2, "ring deeper than the score commits can track");
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
-  static constexpr int kSmemTiles = (2 + kStages) * kTileBytes;
-  static constexpr int kSmemBytesRaw = 1024 + kSmemTiles + 1024;
-  // Keep one CTA per SM so that the 512-column TMEM allocation never waits on a sibling CTA.
-  static constexpr int kSmemBytes = kSmemBytesRaw > 120 * 1024 ? kSmemBytesRaw : 120 * 1024;
+  static constexpr uint32_t kColO = 0, kColS = 128;  // score buffer b at kColS + 128 b
+  static constexpr int kSmemTiles = (kQBufs + kStages) * kTileBytes;
+  static constexpr int kSmemBytes = 1024 + kSmemTiles + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory");
   static constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(128, 128, false);
   static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, true);
 };
 
-constexpr int kNumThreads = 320;  // 8 SiLU warps + producer + MMA issuer
+constexpr int kNumThreads = 448;  // 8 SiLU warps + producer + MMA issuer + 4 epilogue warps
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;       // issues every MMA and owns the TMEM allocation
+constexpr int kEpiWarp0 = 10;     // first of the four epilogue warps
+constexpr int kSlots = 4;         // work-item slots between the producer and the other roles
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s per wait
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s per drain wait on the abort path
 
@@ -92,13 +117,14 @@ struct FwdParams {
 
 template <int kStages>
 struct SmemCtl {
-  uint64_t q_full, q_empty;
-  uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
-  uint64_t sched_full[2], sched_empty[2];
+  uint64_t q_empty[2];
+  uint64_t g_ready[kGroupBars];  // group g: its Q/V/K bytes and P_{g-3} are in
+  uint64_t s_full[kSCommits];
+  uint64_t o_full, o_empty;
+  uint64_t sched_full[kSlots], sched_empty[kSlots];
   uint64_t drain;
   // work slot: valid, h, kv_start, q_row0, pos0, nrows, L, U
-  int32_t slot[2][8];
+  int32_t slot[kSlots][8];
   uint32_t tmem_base;
   int32_t abort_flag;
 };
@@ -120,14 +146,24 @@ __device__ __forceinline__ Work read_slot(const volatile int32_t* s) {
   return w;
 }
 
-// Slow path of wait_bounded: spins until the phase completes, the CTA aborts, or the time limit.
+// Limits below this are test limits: their waits poll instead of suspending in try_wait, whose
+// suspension may last until the phase completes, so that the clock is read every few clocks.
+constexpr uint64_t kPollBelowNs = 1000000ull;
+
+__device__ __forceinline__ uint32_t suspend_hint(uint64_t limit_ns) {
+  return limit_ns < 0xffffffffull ? (uint32_t)limit_ns : 0xffffffffu;
+}
+
+// Slow path of wait_bounded: waits until the phase completes, the CTA aborts, or the time limit.
 // Each try_wait may itself suspend the thread for a while, so the flag and the clock are checked
 // after every attempt.
 __device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag,
                                                unsigned* err, uint64_t limit_ns) {
   const uint64_t t0 = ptx::globaltimer_ns();
+  const bool poll = limit_ns < kPollBelowNs;
   while (true) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (poll ? ptx::mbar_test_wait(bar, parity) : ptx::mbar_try_wait_for(bar, parity, suspend_hint(limit_ns)))
+      return true;
     if (*abort_flag) return false;
     if (ptx::globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
@@ -138,17 +174,19 @@ __device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity, vo
 }
 
 // Waits for phase `parity` of `bar`; false if the CTA is aborting or this wait timed out.  The
-// first test is inline: a call right after a burst of MMAs stalls the issuing warp.
+// first try is inline (a call right after a burst of MMAs stalls the issuing warp) and may
+// suspend the thread until the phase completes; a wait with a test limit goes straight to the
+// polling slow path instead.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag,
                                              unsigned* err, uint64_t limit_ns = kWaitLimitNs) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
+  if (limit_ns >= kPollBelowNs && ptx::mbar_try_wait_for(bar, parity, 0xffffffffu)) return true;
   return wait_bounded_slow(bar, parity, abort_flag, err, limit_ns);
 }
 
 // Abort-path drain: waits for phase `parity` of `bar` for at most kDrainLimitNs.
 __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = ptx::globaltimer_ns();
-  while (!ptx::mbar_try_wait(bar, parity))
+  while (!ptx::mbar_try_wait_for(bar, parity, (uint32_t)kDrainLimitNs))
     if (ptx::globaltimer_ns() - t0 > kDrainLimitNs) return;
 }
 
@@ -203,6 +241,18 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t tad
   ptx::tmem_st16(taddr_s + kChunk * 16, pk);
 }
 
+// Loads run K_0 K_1 K_2 | V_0 K_3 | V_1 K_4 | ... in the order the MMA warp consumes them, so load
+// e < 3 is consumed by group e and load e >= 3 by group (e + 3) / 2.  (The closing one to three V
+// loads of the CTA, consumed by P.V-only groups, are never looked up: no load follows them by a
+// whole ring.)
+__device__ __forceinline__ int group_of_load(int e) { return e < 3 ? e : (e + 3) >> 1; }
+
+// Rows of sub-item hh of a work item (query rows [128 hh, 128 hh + 128)); <= 0 if it has none.
+__device__ __forceinline__ int sub_rows(const Work& w, int hh) {
+  const int r = w.nrows - hh * kTileRows;
+  return r < kTileRows ? r : kTileRows;
+}
+
 template <int D, bool kRab>
 __global__ void __launch_bounds__(kNumThreads, 1)
     hstu_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -213,8 +263,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   const uint32_t raw_addr = ptx::smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
   const uint32_t sbase = ptx::smem_addr(smem);
-  const uint32_t sQ = sbase;                                  // 2 tiles
-  const uint32_t sKV = sbase + 2 * Cfg::kTileBytes;           // kStages tiles
+  const uint32_t sQ = sbase;                                   // kQBufs tiles
+  const uint32_t sKV = sbase + Cfg::kQBufs * Cfg::kTileBytes;  // kStages tiles
   auto* ctl = reinterpret_cast<SmemCtl<Cfg::kStages>*>(smem + Cfg::kSmemTiles);
   volatile int32_t* abort_flag = &ctl->abort_flag;
 
@@ -224,19 +274,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   auto bar = [](const uint64_t& b) { return ptx::smem_addr(&b); };
 
   if (warp == kProducerWarp && lane == 0) {
-    ptx::mbar_init(bar(ctl->q_full), 1);
-    ptx::mbar_init(bar(ctl->q_empty), 1);
-    for (int s = 0; s < Cfg::kStages; ++s) {
-      ptx::mbar_init(bar(ctl->kv_full[s]), 1);
-      ptx::mbar_init(bar(ctl->kv_empty[s]), 1);
-    }
-    for (int h = 0; h < 2; ++h) {
-      ptx::mbar_init(bar(ctl->s_full[h]), 1);
-      ptx::mbar_init(bar(ctl->p_full[h]), 4);   // one arrival per SiLU warp
-      ptx::mbar_init(bar(ctl->o_full[h]), 1);
-      ptx::mbar_init(bar(ctl->o_empty[h]), 4);
-      ptx::mbar_init(bar(ctl->sched_full[h]), 1);
-      ptx::mbar_init(bar(ctl->sched_empty[h]), 1 + 8);
+    for (int i = 0; i < 2; ++i) ptx::mbar_init(bar(ctl->q_empty[i]), 1);
+    // The producer's expect-tx arrival plus one arrival per warp of the SiLU warpgroup.
+    for (int i = 0; i < kGroupBars; ++i) ptx::mbar_init(bar(ctl->g_ready[i]), 1 + 4);
+    for (int b = 0; b < kSCommits; ++b) ptx::mbar_init(bar(ctl->s_full[b]), 1);
+    ptx::mbar_init(bar(ctl->o_full), 1);
+    ptx::mbar_init(bar(ctl->o_empty), 4);      // one arrival per epilogue warp
+    for (int s = 0; s < kSlots; ++s) {
+      ptx::mbar_init(bar(ctl->sched_full[s]), 1);
+      ptx::mbar_init(bar(ctl->sched_empty[s]), 1 + 8 + 4);  // MMA, SiLU and epilogue warps
     }
     ptx::mbar_init(bar(ctl->drain), 1);
     ctl->abort_flag = 0;
@@ -262,12 +308,26 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       asm volatile("griddepcontrol.wait;" ::: "memory");
       const int M = *p.num_items;
       int slot = 0;
-      uint32_t sched_empty_par[2] = {1u, 1u};
-      uint32_t q_empty_par = 1u;
-      int stage = 0;
-      uint32_t kv_phase = 0;
+      uint32_t sched_empty_par = (1u << kSlots) - 1u;  // bit s: parity of slot s's next wait
+      int sub = 0;        // sub-items whose Q load was issued
+      int j = 0;          // K/V loads issued
+      int g = 0;          // score tiles (groups with an S) armed
+      int armed_hi = 0;   // one past the highest group index armed
+      // V rows and heads of tiles g-3, g-2, g-1.
+      int vrow0 = 0, vrow1 = 0, vrow2 = 0, vh0 = 0, vh1 = 0, vh2 = 0;
       bool ok = true;
-      int issued_q = 0, issued_kv = 0;
+      // True once ring slot e mod kStages is free: the group that consumed the slot's previous
+      // tile (load e - kStages) has completed.
+      auto slot_free = [&](int e) {
+        if (e < Cfg::kStages) return true;
+        const int G = group_of_load(e - Cfg::kStages);
+        return wait_bounded(bar(ctl->s_full[G % kSCommits]), (uint32_t)((G / kSCommits) & 1), abort_flag, p.err,
+                            p.wait_limit_ns);
+      };
+      auto tma_tile = [&](const CUtensorMap* tm, uint32_t dst, uint32_t rb, int col0, int row) {
+        for (int blk = 0; blk < Cfg::kBlocks; ++blk)
+          ptx::tma_load_2d(dst + blk * Cfg::kBlockBytes, tm, rb, col0 + blk * Cfg::kBlockElems, row);
+      };
       while (ok) {
         const int idx = atomicAdd(p.work_counter, 1);
         Work w{};
@@ -286,53 +346,80 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const int rows = (w.L - c) - pair * kPairRows;
           w.nrows = rows < kPairRows ? rows : kPairRows;
         }
-        if (!wait_bounded(bar(ctl->sched_empty[slot]), sched_empty_par[slot], abort_flag, p.err, p.wait_limit_ns)) break;
-        sched_empty_par[slot] ^= 1u;
+        if (!wait_bounded(bar(ctl->sched_empty[slot]), (sched_empty_par >> slot) & 1u, abort_flag, p.err,
+                          p.wait_limit_ns)) {
+          ok = false;
+          break;
+        }
+        sched_empty_par ^= 1u << slot;
         volatile int32_t* s = ctl->slot[slot];
         s[0] = w.valid; s[1] = w.h; s[2] = w.kv_start; s[3] = w.q_row0;
         s[4] = w.pos0; s[5] = w.nrows; s[6] = w.L; s[7] = w.U;
         ptx::mbar_arrive(bar(ctl->sched_full[slot]));
-        slot ^= 1;
+        slot = (slot + 1) & (kSlots - 1);
         if (!w.valid) break;
 
-        const TileRange un = key_tiles(w.pos0, w.pos0 + w.nrows, w.U);
-        const int n_u = tile_count(un);
-        if (!wait_bounded(bar(ctl->q_empty), q_empty_par, abort_flag, p.err, p.wait_limit_ns)) break;
-        q_empty_par ^= 1u;
-        ptx::mbar_arrive_expect_tx(bar(ctl->q_full), 2 * Cfg::kTileBytes);
-        for (int hh = 0; hh < 2; ++hh)
-          for (int blk = 0; blk < Cfg::kBlocks; ++blk)
-            ptx::tma_load_2d(sQ + hh * Cfg::kTileBytes + blk * Cfg::kBlockBytes, &tm_q, bar(ctl->q_full),
-                             w.h * D + blk * Cfg::kBlockElems, w.q_row0 + hh * kTileRows);
-        ++issued_q;
-        for (int i = 0; i < n_u && ok; ++i) {
-          const int row = w.kv_start + tile_at(un, i) * kTileRows;
-          for (int kv = 0; kv < 2; ++kv) {
-            if (!wait_bounded(bar(ctl->kv_empty[stage]), kv_phase ^ 1u, abort_flag, p.err, p.wait_limit_ns)) {
-              ok = false;
-              break;
+        for (int hh = 0; hh < 2 && ok; ++hh) {
+          const int nr = sub_rows(w, hh);
+          if (nr <= 0) break;
+          const int lo = hh * kTileRows;
+          const TileRange r = key_tiles(w.pos0 + lo, w.pos0 + lo + nr, w.U);
+          const int n = tile_count(r);
+          const int qb = sub & 1;
+          if (!wait_bounded(bar(ctl->q_empty[qb]), (uint32_t)(((sub >> 1) & 1) ^ 1), abort_flag, p.err,
+                            p.wait_limit_ns)) {
+            ok = false;
+            break;
+          }
+          for (int k = 0; k < n; ++k) {
+            // Group g reads V_{g-3} (load j) and K_g (load j+1), or K_g alone for g < 3, and Q on
+            // a sub-item's first tile; all of them land on the group's ready barrier.
+            const bool has_v = g >= 3;
+            if (!slot_free(j) || (has_v && !slot_free(j + 1))) { ok = false; break; }
+            const int krow = w.kv_start + tile_at(r, k) * kTileRows;
+            const uint32_t rb = bar(ctl->g_ready[g & (kGroupBars - 1)]);
+            ptx::mbar_arrive_expect_tx(rb, Cfg::kTileBytes * (1 + (has_v ? 1 : 0) + (k == 0 ? 1 : 0)));
+            if (!has_v)  // no P.V in this group: stand in for the SiLU warps' arrivals
+              for (int a = 0; a < 4; ++a) ptx::mbar_arrive(rb);
+            if (k == 0) {
+              tma_tile(&tm_q, sQ + qb * Cfg::kTileBytes, rb, w.h * D, w.q_row0 + lo);
+              ++sub;
             }
-            const uint32_t fb = bar(ctl->kv_full[stage]);
-            ptx::mbar_arrive_expect_tx(fb, Cfg::kTileBytes);
-            const CUtensorMap* tm = kv ? &tm_v : &tm_k;
-            for (int blk = 0; blk < Cfg::kBlocks; ++blk)
-              ptx::tma_load_2d(sKV + stage * Cfg::kTileBytes + blk * Cfg::kBlockBytes, tm, fb,
-                               w.h * D + blk * Cfg::kBlockElems, row);
-            ++issued_kv;
-            if (++stage == Cfg::kStages) {
-              stage = 0;
-              kv_phase ^= 1u;
+            if (has_v) {
+              tma_tile(&tm_v, sKV + (j % Cfg::kStages) * Cfg::kTileBytes, rb, vh0 * D, vrow0);
+              ++j;
             }
+            tma_tile(&tm_k, sKV + (j % Cfg::kStages) * Cfg::kTileBytes, rb, w.h * D, krow);
+            ++j;
+            vrow0 = vrow1; vh0 = vh1;
+            vrow1 = vrow2; vh1 = vh2;
+            vrow2 = krow;  vh2 = w.h;
+            armed_hi = ++g;
           }
         }
       }
+      // The closing groups t + 3 carry the V tiles of the last (up to) three score tiles t.
+      for (int t = (g >= 3 ? g - 3 : 0); t < g && ok; ++t) {
+        const int i = t - g + 3;  // 0, 1, 2 <-> tiles g-3, g-2, g-1
+        const int row = i == 0 ? vrow0 : (i == 1 ? vrow1 : vrow2);
+        const int h = i == 0 ? vh0 : (i == 1 ? vh1 : vh2);
+        if (!slot_free(j)) { ok = false; break; }
+        const uint32_t rb = bar(ctl->g_ready[(t + 3) & (kGroupBars - 1)]);
+        ptx::mbar_arrive_expect_tx(rb, Cfg::kTileBytes);
+        tma_tile(&tm_v, sKV + (j % Cfg::kStages) * Cfg::kTileBytes, rb, h * D, row);
+        ++j;
+        armed_hi = t + 4;
+      }
       if (*abort_flag) {
-        // Let every copy this CTA started land before its shared memory is released.
-        for (int k = 1; k <= Cfg::kStages && k <= issued_kv; ++k) {
-          const int pos = issued_kv - k;  // load index
-          drain_wait(bar(ctl->kv_full[pos % Cfg::kStages]), (uint32_t)((pos / Cfg::kStages) & 1));
+        // Let every copy this CTA started land before its shared memory is released: each group
+        // barrier still in use gets the SiLU arrivals that may never come (extra ones only spill
+        // into a phase nobody waits for), then its bytes are awaited.
+        for (int x = armed_hi > kGroupBars ? armed_hi - kGroupBars : 0; x < armed_hi; ++x) {
+          if (x >= g && x < 3) continue;  // group indices never used when the CTA had < 3 tiles
+          const uint32_t rb = bar(ctl->g_ready[x & (kGroupBars - 1)]);
+          for (int a = 0; a < 4; ++a) ptx::mbar_arrive(rb);
+          drain_wait(rb, (uint32_t)((x / kGroupBars) & 1));
         }
-        if (issued_q > 0) drain_wait(bar(ctl->q_full), (uint32_t)((issued_q - 1) & 1));
       }
     }
     __syncwarp();
@@ -341,6 +428,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // The whole warp runs this loop in step, so the control flow is uniform and the descriptors
     // and TMEM addresses stay in uniform registers; lane 0 alone issues the tcgen05 instructions
     // (the *_lead forms), so every MMA and commit comes from one thread, as commit tracking needs.
+    // The loop keeps its ring slot, buffer and barrier indices as running counters: every
+    // instruction between two MMA bursts is tensor-core idle time.
     const uint32_t lead = (lane == 0) ? 1u : 0u;
     // Waits are taken by every lane and the outcome is made warp-uniform.
     auto wait_all = [&](uint32_t b, uint32_t par) {
@@ -351,242 +440,257 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const uint64_t dk0 = ptx::smem_desc(sKV, 16, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
     const uint64_t dv0 = ptx::smem_desc(sKV, Cfg::kBlockBytes, 8 * Cfg::kRowBytes, Cfg::kSwizzle);
     int slot = 0;
-    uint32_t sched_full_par[2] = {0u, 0u};
-    uint32_t q_full_par = 0u;
-    uint32_t p_full_par[2] = {0u, 0u};
-    uint32_t o_empty_par[2] = {1u, 1u};
-    int stage = 0;
-    uint32_t kv_phase = 0;
+    uint32_t sched_full_par = 0u;  // bit s: parity of slot s's next wait
+    int sub = 0;
+    int g = 0;               // groups with an S issued
+    int st = 0;              // ring slot of the next tile to consume
+    uint32_t b3 = 0;         // g mod 3: score buffer of S_g, and of P_{g-3}
+    int c6 = 0;              // g mod kSCommits: barrier of S_g's commit
+    int r8 = 0;              // g mod kGroupBars: ready barrier of group g
+    uint32_t rpar = 0u;      // parity of that barrier's phase for group g
+    uint32_t o_empty_par = 1u;
+    // Tiles g-3, g-2, g-1: bit 0 = first tile of its sub-item, bit 1 = last tile of its sub-item.
+    uint32_t f0 = 0, f1 = 0, f2 = 0;
     bool ok = true;
+    // O += P V for a tile whose P is in score buffer pb and whose V is in ring slot vs (its group's
+    // ready barrier already waited).  A sub-item's first tile starts O afresh once the epilogue
+    // has read the previous O; its last one commits O to the epilogue.
+    auto issue_pv = [&](uint32_t pb, int vs, uint32_t flags) {
+      if (flags & 1u) {
+        if (!wait_all(bar(ctl->o_empty), o_empty_par)) return false;
+        o_empty_par ^= 1u;
+      }
+      ptx::tc_fence_after();
+      const uint64_t dv = dv0 + ((vs * Cfg::kTileBytes) >> 4);
+      const uint32_t colP = Cfg::kColS + 128u * pb;
+#pragma unroll
+      for (int ks = 0; ks < kTileRows / 16; ++ks)
+        ptx::mma_ts_lead(lead, tmem + Cfg::kColO, tmem + colP + ks * 8, dv + ((ks * 16 * Cfg::kRowBytes) >> 4),
+                         Cfg::kIdescPV, ((flags & 1u) && ks == 0) ? 0u : 1u);
+      if (flags & 2u) ptx::mma_commit_lead(lead, bar(ctl->o_full));
+      return true;
+    };
+    auto next_slot = [](int s) { return s + 1 == Cfg::kStages ? 0 : s + 1; };
     while (ok) {
-      if (!wait_all(bar(ctl->sched_full[slot]), sched_full_par[slot])) break;
-      sched_full_par[slot] ^= 1u;
+      if (!wait_all(bar(ctl->sched_full[slot]), (sched_full_par >> slot) & 1u)) {
+        ok = false;
+        break;
+      }
+      sched_full_par ^= 1u << slot;
       const Work w = read_slot(ctl->slot[slot]);
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(ctl->sched_empty[slot]));
-      slot ^= 1;
+      slot = (slot + 1) & (kSlots - 1);
       if (!w.valid) break;
 
-      const TileRange un = key_tiles(w.pos0, w.pos0 + w.nrows, w.U);
-      TileRange hr[2];
-      int remaining[2];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
+      for (int hh = 0; hh < 2 && ok; ++hh) {
+        const int nr = sub_rows(w, hh);
+        if (nr <= 0) break;
         const int lo = hh * kTileRows;
-        const int hi = w.nrows < lo + kTileRows ? w.nrows : lo + kTileRows;
-        hr[hh] = key_tiles(w.pos0 + lo, w.pos0 + (hi > lo ? hi : lo), w.U);
-        remaining[hh] = tile_count(hr[hh]);
-      }
-      const int n_u = tile_count(un);
-      if (!wait_all(bar(ctl->q_full), q_full_par)) break;
-      q_full_par ^= 1u;
-      ptx::tc_fence_after();
-
-      bool pend[2] = {false, false};
-      bool first[2] = {true, true};
-      int prev_vst = 0;
-      uint32_t prev_vph = 0;
-      // Step i, per half in turn: the P.V of the previous key tile (if that half used it), then
-      // the scores of key tile i (if that half needs it).  The tensor pipe therefore alternates
-      // [P.V_0, S_0], [P.V_1, S_1], and one half's SiLU overlaps the other half's MMAs.  The
-      // extra last step only drains the P.V.
-      for (int i = 0; i <= n_u; ++i) {
-        const bool last = (i == n_u);
-        int t = 0, kst = 0, vst = 0;
-        uint32_t kph = 0, vph = 0;
-        if (!last) {
-          t = tile_at(un, i);
-          kst = stage;
-          kph = kv_phase;
-          if (++stage == Cfg::kStages) { stage = 0; kv_phase ^= 1u; }
-          vst = stage;
-          vph = kv_phase;
-          if (++stage == Cfg::kStages) { stage = 0; kv_phase ^= 1u; }
-        }
-        bool k_waited = false, v_waited = false;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const uint32_t colS = hh ? Cfg::kColS1 : Cfg::kColS0;
-          if (pend[hh]) {
-            ok = wait_all(bar(ctl->p_full[hh]), p_full_par[hh]) &&
-                 (v_waited || wait_all(bar(ctl->kv_full[prev_vst]), prev_vph)) &&
-                 (!first[hh] || wait_all(bar(ctl->o_empty[hh]), o_empty_par[hh]));
-            if (!ok) break;
-            v_waited = true;
-            p_full_par[hh] ^= 1u;
-            if (first[hh]) o_empty_par[hh] ^= 1u;
-            ptx::tc_fence_after();
-            const uint64_t dv = dv0 + ((prev_vst * Cfg::kTileBytes) >> 4);
-            const uint32_t colO = hh ? Cfg::kColO1 : Cfg::kColO0;
-#pragma unroll
-            for (int ks = 0; ks < kTileRows / 16; ++ks)
-              ptx::mma_ts_lead(lead, tmem + colO, tmem + colS + ks * 8, dv + ((ks * 16 * Cfg::kRowBytes) >> 4),
-                               Cfg::kIdescPV, (first[hh] && ks == 0) ? 0u : 1u);
-            first[hh] = false;
-            pend[hh] = false;
-            if (--remaining[hh] == 0) ptx::mma_commit_lead(lead, bar(ctl->o_full[hh]));
+        const TileRange r = key_tiles(w.pos0 + lo, w.pos0 + lo + nr, w.U);
+        const int n = tile_count(r);
+        const int qb = sub & 1;
+        const uint64_t dq = dq0 + ((qb * Cfg::kTileBytes) >> 4);
+        for (int k = 0; k < n; ++k) {
+          // Group g: once its tiles and P_{g-3} are in, the P.V of tile g-3, then the scores of
+          // tile g into buffer g mod 3, then one commit.
+          if (!wait_all(bar(ctl->g_ready[r8]), rpar)) { ok = false; break; }
+          ptx::tc_fence_after();
+          if (g >= 3) {
+            if (!issue_pv(b3, st, f0)) { ok = false; break; }
+            st = next_slot(st);
           }
-          if (!last && tile_in(hr[hh], t)) {
-            if (!k_waited) {
-              if (!wait_all(bar(ctl->kv_full[kst]), kph)) { ok = false; break; }
-              ptx::tc_fence_after();
-              k_waited = true;
-            }
-            const uint64_t dq = dq0 + ((hh * Cfg::kTileBytes) >> 4);
-            const uint64_t dk = dk0 + ((kst * Cfg::kTileBytes) >> 4);
+          const uint64_t dk = dk0 + ((st * Cfg::kTileBytes) >> 4);
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-              const uint32_t off =
-                  (ks / Cfg::kKStepsPerBlock) * Cfg::kBlockBytes + (ks % Cfg::kKStepsPerBlock) * 32;
-              ptx::mma_ss_lead(lead, tmem + colS, dq + (off >> 4), dk + (off >> 4), Cfg::kIdescQK,
-                               ks > 0 ? 1u : 0u);
-            }
-            ptx::mma_commit_lead(lead, bar(ctl->s_full[hh]));
-            pend[hh] = true;
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off =
+                (ks / Cfg::kKStepsPerBlock) * Cfg::kBlockBytes + (ks % Cfg::kKStepsPerBlock) * 32;
+            ptx::mma_ss_lead(lead, tmem + Cfg::kColS + 128u * b3, dq + (off >> 4), dk + (off >> 4), Cfg::kIdescQK,
+                             ks > 0 ? 1u : 0u);
           }
+          st = next_slot(st);
+          ptx::mma_commit_lead(lead, bar(ctl->s_full[c6]));
+          if (k == n - 1) ptx::mma_commit_lead(lead, bar(ctl->q_empty[qb]));  // Q: free after its last S
+          f0 = f1;
+          f1 = f2;
+          f2 = (k == 0 ? 1u : 0u) | (k == n - 1 ? 2u : 0u);
+          ++g;
+          b3 = (b3 == 2u) ? 0u : b3 + 1u;
+          c6 = (c6 == kSCommits - 1) ? 0 : c6 + 1;
+          r8 = (r8 + 1) & (kGroupBars - 1);
+          if (r8 == 0) rpar ^= 1u;
         }
-        if (!ok) break;
-        if (!last) ptx::mma_commit_lead(lead, bar(ctl->kv_empty[kst]));       // K_t: free after its S MMAs
-        if (i > 0) ptx::mma_commit_lead(lead, bar(ctl->kv_empty[prev_vst]));  // V_{t-1}: free after its P.V
-        if (i == n_u - 1) ptx::mma_commit_lead(lead, bar(ctl->q_empty));      // Q: free after the last S MMA
-        prev_vst = vst;
-        prev_vph = vph;
+        ++sub;
       }
+    }
+    // The closing groups t + 3: the P.V of the last (up to) three tiles t.
+    for (int t = (g >= 3 ? g - 3 : 0); t < g && ok; ++t) {
+      const int i = t - g + 3;  // 0, 1, 2 <-> tiles g-3, g-2, g-1
+      const int x = t + 3;
+      ok = wait_all(bar(ctl->g_ready[x & (kGroupBars - 1)]), (uint32_t)((x / kGroupBars) & 1)) &&
+           issue_pv((uint32_t)(t % 3), st, i == 0 ? f0 : (i == 1 ? f1 : f2));
+      st = next_slot(st);
     }
     // Every MMA lane 0 issued has completed once `drain` flips.
     ptx::mma_commit_lead(lead, bar(ctl->drain));
     drain_wait(bar(ctl->drain), 0u);
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------------ SiLU + epilogue
-    const int hh = warp >> 2;          // half
+  } else if (warp < kProducerWarp) {
+    // ------------------------------------------------------------------ SiLU
+    const int wg = warp >> 2;          // takes the score tiles g with g mod 2 == wg
     const int quarter = warp & 3;      // TMEM lane quarter
-    const int row = quarter * 32 + lane;  // row within the half
+    const int row = quarter * 32 + lane;  // row within the query tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t taddr_s = tmem + lane_off + (hh ? Cfg::kColS1 : Cfg::kColS0);
-    const uint32_t taddr_o = tmem + lane_off + (hh ? Cfg::kColO1 : Cfg::kColO0);
     const float half_alpha = p.half_alpha;
-    const float inv_n = p.inv_n;
     int slot = 0;
-    uint32_t sched_full_par[2] = {0u, 0u};
-    uint32_t s_full_par = 0u, o_full_par = 0u;
+    uint32_t sched_full_par = 0u;
+    int g = 0;
     bool ok = true;
     while (ok) {
-      ok = wait_bounded(bar(ctl->sched_full[slot]), sched_full_par[slot], abort_flag, p.err, p.wait_limit_ns);
+      ok = wait_bounded(bar(ctl->sched_full[slot]), (sched_full_par >> slot) & 1u, abort_flag, p.err,
+                        p.wait_limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      sched_full_par[slot] ^= 1u;
+      sched_full_par ^= 1u << slot;
       const Work w = read_slot(ctl->slot[slot]);
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(ctl->sched_empty[slot]));
-      slot ^= 1;
+      slot = (slot + 1) & (kSlots - 1);
       if (!w.valid) break;
 
-      const int lo = hh * kTileRows;
-      const int nr = (w.nrows - lo) < kTileRows ? (w.nrows - lo) : kTileRows;
-      if (nr <= 0) continue;
-      const int p0 = w.pos0 + lo;
-      const TileRange r = key_tiles(p0, p0 + nr, w.U);
-      const int n = tile_count(r);
-      const int i_pos = p0 + row;                      // this thread's query position
-      const int lim_abs = (i_pos < w.U) ? i_pos + 1 : w.U;  // keys [0, lim_abs) visible, plus self
       const float* rab_row = kRab ? p.rab + (size_t)w.h * p.rab_len : nullptr;
       const int rab_max = kRab ? p.rab_len - 1 : 0;
-      for (int k = 0; k < n; ++k) {
-        const int j0 = tile_at(r, k) * kTileRows;
-        ok = wait_bounded(bar(ctl->s_full[hh]), s_full_par, abort_flag, p.err, p.wait_limit_ns);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        s_full_par ^= 1u;
-        ptx::tc_fence_after();
-        const bool full = (j0 + kTileRows <= w.U) && (j0 + kTileRows <= p0 + 1);
-        const int lim = lim_abs - j0;
-        const int self = i_pos - j0;
-        const int rel0 = i_pos - j0;
-        // 32-column chunks: the load of chunk c+1 is in flight while chunk c is computed.
-        if constexpr (kRab) {
-          // The bias reads need registers the next chunk's load would hold: one chunk at a time.
-          uint32_t ra[32];
-          ptx::tmem_ld32(taddr_s + 0, ra);
-          ptx::tmem_ld_wait(ra);
-          silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-          ptx::tmem_ld32(taddr_s + 32, ra);
-          ptx::tmem_ld_wait(ra);
-          silu_chunk<1, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-          ptx::tmem_ld32(taddr_s + 64, ra);
-          ptx::tmem_ld_wait(ra);
-          silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-          ptx::tmem_ld32(taddr_s + 96, ra);
-          ptx::tmem_ld_wait(ra);
-          silu_chunk<3, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-        } else {
-          uint32_t ra[32], rb[32];
-          ptx::tmem_ld32(taddr_s + 0, ra);
-          ptx::tmem_ld_wait(ra);
-          ptx::tmem_ld32(taddr_s + 32, rb);
-          silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-          ptx::tmem_ld_wait(rb);
-          ptx::tmem_ld32(taddr_s + 64, ra);
-          silu_chunk<1, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-          ptx::tmem_ld_wait(ra);
-          ptx::tmem_ld32(taddr_s + 96, rb);
-          silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-          ptx::tmem_ld_wait(rb);
-          silu_chunk<3, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+      for (int hh = 0; hh < 2 && ok; ++hh) {
+        const int nr = sub_rows(w, hh);
+        if (nr <= 0) break;
+        const int p0 = w.pos0 + hh * kTileRows;
+        const TileRange r = key_tiles(p0, p0 + nr, w.U);
+        const int n = tile_count(r);
+        const int i_pos = p0 + row;                           // this thread's query position
+        const int lim_abs = (i_pos < w.U) ? i_pos + 1 : w.U;  // keys [0, lim_abs) visible, plus self
+        for (int k = (g + wg) & 1; k < n; k += 2) {
+          const int gt = g + k;
+          const int b = gt % 3;
+          const uint32_t taddr_s = tmem + lane_off + Cfg::kColS + 128u * b;
+          ok = wait_bounded(bar(ctl->s_full[gt % kSCommits]), (uint32_t)((gt / kSCommits) & 1), abort_flag, p.err,
+                            p.wait_limit_ns);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          const int j0 = tile_at(r, k) * kTileRows;
+          const bool full = (j0 + kTileRows <= w.U) && (j0 + kTileRows <= p0 + 1);
+          const int lim = lim_abs - j0;
+          const int self = i_pos - j0;
+          const int rel0 = i_pos - j0;
+          // 32-column chunks: the load of chunk c+1 is in flight while chunk c is computed.
+          if constexpr (kRab) {
+            // The bias reads need registers the next chunk's load would hold: one chunk at a time.
+            uint32_t ra[32];
+            ptx::tmem_ld32(taddr_s + 0, ra);
+            ptx::tmem_ld_wait(ra);
+            silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+            ptx::tmem_ld32(taddr_s + 32, ra);
+            ptx::tmem_ld_wait(ra);
+            silu_chunk<1, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+            ptx::tmem_ld32(taddr_s + 64, ra);
+            ptx::tmem_ld_wait(ra);
+            silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+            ptx::tmem_ld32(taddr_s + 96, ra);
+            ptx::tmem_ld_wait(ra);
+            silu_chunk<3, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          } else {
+            uint32_t ra[32], rb[32];
+            ptx::tmem_ld32(taddr_s + 0, ra);
+            ptx::tmem_ld_wait(ra);
+            ptx::tmem_ld32(taddr_s + 32, rb);
+            silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+            ptx::tmem_ld_wait(rb);
+            ptx::tmem_ld32(taddr_s + 64, ra);
+            silu_chunk<1, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+            ptx::tmem_ld_wait(ra);
+            ptx::tmem_ld32(taddr_s + 96, rb);
+            silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+            ptx::tmem_ld_wait(rb);
+            silu_chunk<3, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          }
+          ptx::tmem_st_wait();
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bar(ctl->g_ready[(gt + 3) & (kGroupBars - 1)]));  // P_gt, for group gt+3
         }
-        ptx::tmem_st_wait();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(ctl->p_full[hh]));
+        g += n;
       }
-      if (!ok) break;
-      // Epilogue: O_h * (1/N) -> bf16 -> out rows that exist.
-      ok = wait_bounded(bar(ctl->o_full[hh]), o_full_par, abort_flag, p.err, p.wait_limit_ns);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;         // TMEM lane quarter
+    const int row = quarter * 32 + lane;  // row within the query tile
+    const uint32_t taddr_o = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + Cfg::kColO;
+    const float inv_n = p.inv_n;
+    int slot = 0;
+    uint32_t sched_full_par = 0u, o_full_par = 0u;
+    bool ok = true;
+    while (ok) {
+      ok = wait_bounded(bar(ctl->sched_full[slot]), (sched_full_par >> slot) & 1u, abort_flag, p.err,
+                        p.wait_limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      o_full_par ^= 1u;
-      ptx::tc_fence_after();
-      const size_t orow = (size_t)(w.q_row0 + lo + row);
-      __nv_bfloat16* dst = p.out + orow * p.out_ld + (size_t)w.h * D;
+      sched_full_par ^= 1u << slot;
+      const Work w = read_slot(ctl->slot[slot]);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(ctl->sched_empty[slot]));
+      slot = (slot + 1) & (kSlots - 1);
+      if (!w.valid) break;
+
+      for (int hh = 0; hh < 2 && ok; ++hh) {
+        const int nr = sub_rows(w, hh);
+        if (nr <= 0) break;
+        ok = wait_bounded(bar(ctl->o_full), o_full_par, abort_flag, p.err, p.wait_limit_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        o_full_par ^= 1u;
+        ptx::tc_fence_after();
+        // O * (1/N) -> bf16 pairs in registers; O is then released to the next sub-item's P.V.
+        uint32_t a[D / 2];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ro[32];
-        ptx::tmem_ld32(taddr_o + c * 32, ro);
-        ptx::tmem_ld_wait(ro);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ro[32];
+          ptx::tmem_ld32(taddr_o + c * 32, ro);
+          ptx::tmem_ld_wait(ro);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            a[c * 16 + e] = pack_bf16x2(__uint_as_float(ro[2 * e]) * inv_n, __uint_as_float(ro[2 * e + 1]) * inv_n);
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(ctl->o_empty));
         if (row < nr) {
-          uint4 a4[4];
+          const size_t orow = (size_t)(w.q_row0 + hh * kTileRows + row);
+          const size_t col = (size_t)w.h * D;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + orow * p.out_ld + col);
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            a4[q4].x = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 0]) * inv_n, __uint_as_float(ro[q4 * 8 + 1]) * inv_n);
-            a4[q4].y = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 2]) * inv_n, __uint_as_float(ro[q4 * 8 + 3]) * inv_n);
-            a4[q4].z = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 4]) * inv_n, __uint_as_float(ro[q4 * 8 + 5]) * inv_n);
-            a4[q4].w = pack_bf16x2(__uint_as_float(ro[q4 * 8 + 6]) * inv_n, __uint_as_float(ro[q4 * 8 + 7]) * inv_n);
-            reinterpret_cast<uint4*>(dst + c * 32)[q4] = a4[q4];
-          }
+          for (int q4 = 0; q4 < D / 8; ++q4)
+            dst[q4] = make_uint4(a[4 * q4], a[4 * q4 + 1], a[4 * q4 + 2], a[4 * q4 + 3]);
           if (p.gate != nullptr) {
             // Layer epilogue: the gate row U, a copy of it and U * A, beside A in the next
             // projection's input.
-            const size_t col = (size_t)w.h * D + c * 32;
             const uint4* u4 = reinterpret_cast<const uint4*>(p.gate + orow * p.gate_ld + col);
             uint4* cp4 = reinterpret_cast<uint4*>(p.gate_copy + orow * p.out_ld + col);
             uint4* pr4 = reinterpret_cast<uint4*>(p.gate_prod + orow * p.out_ld + col);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int q4 = 0; q4 < D / 8; ++q4) {
               const uint4 u = u4[q4];
               cp4[q4] = u;
               uint4 pr;
-              pr.x = mul_bf16x2(u.x, a4[q4].x);
-              pr.y = mul_bf16x2(u.y, a4[q4].y);
-              pr.z = mul_bf16x2(u.z, a4[q4].z);
-              pr.w = mul_bf16x2(u.w, a4[q4].w);
+              pr.x = mul_bf16x2(u.x, a[4 * q4]);
+              pr.y = mul_bf16x2(u.y, a[4 * q4 + 1]);
+              pr.z = mul_bf16x2(u.z, a[4 * q4 + 2]);
+              pr.w = mul_bf16x2(u.w, a[4 * q4 + 3]);
               pr4[q4] = pr;
             }
           }
         }
       }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(ctl->o_empty[hh]));
     }
   }
 
