@@ -212,12 +212,16 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t tad
                                            bool full, int lim, int self, const float* rab_row, int rel0,
                                            int rab_max) {
   uint32_t pk[16];
+  // Columns are taken in pairs on the two-wide FMA pipe: h = s * alpha/2 and p = h * tanh(h) + h,
+  // bit-identical to the scalar forms.
+  const uint64_t ha2 = ptx::f32x2(half_alpha, half_alpha);
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
-    const float h0 = __uint_as_float(r[2 * e]) * half_alpha;
-    const float h1 = __uint_as_float(r[2 * e + 1]) * half_alpha;
-    float p0 = fmaf(h0, ptx::tanh_approx(h0), h0);
-    float p1 = fmaf(h1, ptx::tanh_approx(h1), h1);
+    const uint64_t h2 = ptx::mul_f32x2(ptx::f32x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), ha2);
+    float h0, h1;
+    ptx::f32x2_split(h2, h0, h1);
+    float p0, p1;
+    ptx::f32x2_split(ptx::fma_f32x2(h2, ptx::f32x2(ptx::tanh_approx(h0), ptx::tanh_approx(h1)), h2), p0, p1);
     if constexpr (kRab) {
       // The chunk's distances run down from hi = rel0 - 32*chunk by one per column.  Inside the
       // table the reads are fixed offsets from one base; otherwise (masked pairs have negative
@@ -582,37 +586,21 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const int lim = lim_abs - j0;
           const int self = i_pos - j0;
           const int rel0 = i_pos - j0;
-          // 32-column chunks: the load of chunk c+1 is in flight while chunk c is computed.
-          if constexpr (kRab) {
-            // The bias reads need registers the next chunk's load would hold: one chunk at a time.
-            uint32_t ra[32];
-            ptx::tmem_ld32(taddr_s + 0, ra);
-            ptx::tmem_ld_wait(ra);
-            silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-            ptx::tmem_ld32(taddr_s + 32, ra);
-            ptx::tmem_ld_wait(ra);
-            silu_chunk<1, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-            ptx::tmem_ld32(taddr_s + 64, ra);
-            ptx::tmem_ld_wait(ra);
-            silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-            ptx::tmem_ld32(taddr_s + 96, ra);
-            ptx::tmem_ld_wait(ra);
-            silu_chunk<3, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-          } else {
-            uint32_t ra[32], rb[32];
-            ptx::tmem_ld32(taddr_s + 0, ra);
-            ptx::tmem_ld_wait(ra);
-            ptx::tmem_ld32(taddr_s + 32, rb);
-            silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-            ptx::tmem_ld_wait(rb);
-            ptx::tmem_ld32(taddr_s + 64, ra);
-            silu_chunk<1, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-            ptx::tmem_ld_wait(ra);
-            ptx::tmem_ld32(taddr_s + 96, rb);
-            silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-            ptx::tmem_ld_wait(rb);
-            silu_chunk<3, kRab>(rb, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
-          }
+          // 32-column chunks, one at a time: the registers a second buffer would take keep the
+          // SiLU free of spills, and the other SiLU warps on the scheduler cover the load latency.
+          uint32_t ra[32];
+          ptx::tmem_ld32(taddr_s + 0, ra);
+          ptx::tmem_ld_wait(ra);
+          silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          ptx::tmem_ld32(taddr_s + 32, ra);
+          ptx::tmem_ld_wait(ra);
+          silu_chunk<1, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          ptx::tmem_ld32(taddr_s + 64, ra);
+          ptx::tmem_ld_wait(ra);
+          silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          ptx::tmem_ld32(taddr_s + 96, ra);
+          ptx::tmem_ld_wait(ra);
+          silu_chunk<3, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
           ptx::tmem_st_wait();
           ptx::tc_fence_before();
           __syncwarp();
