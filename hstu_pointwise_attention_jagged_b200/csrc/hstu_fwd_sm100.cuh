@@ -205,12 +205,28 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
 // SiLU + mask + bf16 pack of 32 score columns [32*chunk, 32*chunk+32) of this thread's row,
 // written as 16 packed columns [16*chunk, 16*chunk+16) of the same TMEM row.
 // lim/self are relative to the tile's first key: key column c is visible iff c < lim || c == self.
-// With kRab, a visible pair also gets rab_row[min(rel0 - c, rab_max)], its query-key distance
-// clipped to the last table entry (rel0 = query position - first key of the tile).
+// With kRab, a visible pair also gets bias[c] (load_bias: rab_row[min(rel0 - c, rab_max)], its
+// query-key distance clipped to the last table entry; rel0 = query position - first key of the
+// tile).
+// The 32 biases of chunk kChunk of this row: column c has distance rel0 - 32*kChunk - c, clipped
+// to [0, rab_max] (negative distances are masked pairs).  The loads are issued together, ahead of
+// the chunk's TMEM load, so their latency is paid once per chunk rather than once per pair.  A
+// warp's load of one column reads 32 consecutive entries (the rows' distances differ by one).
+template <int kChunk>
+__device__ __forceinline__ void load_bias(float (&b)[32], const float* rab_row, int rel0, int rab_max) {
+  const int hi = rel0 - kChunk * 32;
+  if (hi >= 31 && hi <= rab_max) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) b[c] = __ldg(rab_row + hi - c);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) b[c] = __ldg(rab_row + min(max(hi - c, 0), rab_max));
+  }
+}
+
 template <int kChunk, bool kRab>
 __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t taddr_s, float half_alpha,
-                                           bool full, int lim, int self, const float* rab_row, int rel0,
-                                           int rab_max) {
+                                           bool full, int lim, int self, const float (&bias)[32]) {
   uint32_t pk[16];
   // Columns are taken in pairs on the two-wide FMA pipe: h = s * alpha/2 and p = h * tanh(h) + h,
   // bit-identical to the scalar forms.
@@ -223,17 +239,8 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t tad
     float p0, p1;
     ptx::f32x2_split(ptx::fma_f32x2(h2, ptx::f32x2(ptx::tanh_approx(h0), ptx::tanh_approx(h1)), h2), p0, p1);
     if constexpr (kRab) {
-      // The chunk's distances run down from hi = rel0 - 32*chunk by one per column.  Inside the
-      // table the reads are fixed offsets from one base; otherwise (masked pairs have negative
-      // distances, far pairs exceed the table) each index is clamped into it.
-      const int hi = rel0 - kChunk * 32;
-      if (hi >= 31 && hi <= rab_max) {
-        p0 += __ldg(rab_row + hi - 2 * e);
-        p1 += __ldg(rab_row + hi - 2 * e - 1);
-      } else {
-        p0 += __ldg(rab_row + min(max(hi - 2 * e, 0), rab_max));
-        p1 += __ldg(rab_row + min(max(hi - 2 * e - 1, 0), rab_max));
-      }
+      p0 += bias[2 * e];
+      p1 += bias[2 * e + 1];
     }
     if (!full) {
       const int c0 = kChunk * 32 + 2 * e;
@@ -576,31 +583,38 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const int gt = g + k;
           const int b = gt % 3;
           const uint32_t taddr_s = tmem + lane_off + Cfg::kColS + 128u * b;
+          // The first chunk's biases do not depend on S: load them while S is computed.
+          const int j0 = tile_at(r, k) * kTileRows;
+          float bias[32];
+          if constexpr (kRab) load_bias<0>(bias, rab_row, i_pos - j0, rab_max);
           ok = wait_bounded(bar(ctl->s_full[gt % kSCommits]), (uint32_t)((gt / kSCommits) & 1), abort_flag, p.err,
                             p.wait_limit_ns);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           ptx::tc_fence_after();
-          const int j0 = tile_at(r, k) * kTileRows;
           const bool full = (j0 + kTileRows <= w.U) && (j0 + kTileRows <= p0 + 1);
           const int lim = lim_abs - j0;
           const int self = i_pos - j0;
           const int rel0 = i_pos - j0;
           // 32-column chunks, one at a time: the registers a second buffer would take keep the
           // SiLU free of spills, and the other SiLU warps on the scheduler cover the load latency.
+          // With kRab, the next chunk's biases are loaded as soon as the previous chunk is done.
           uint32_t ra[32];
           ptx::tmem_ld32(taddr_s + 0, ra);
           ptx::tmem_ld_wait(ra);
-          silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, bias);
+          if constexpr (kRab) load_bias<1>(bias, rab_row, rel0, rab_max);
           ptx::tmem_ld32(taddr_s + 32, ra);
           ptx::tmem_ld_wait(ra);
-          silu_chunk<1, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          silu_chunk<1, kRab>(ra, taddr_s, half_alpha, full, lim, self, bias);
+          if constexpr (kRab) load_bias<2>(bias, rab_row, rel0, rab_max);
           ptx::tmem_ld32(taddr_s + 64, ra);
           ptx::tmem_ld_wait(ra);
-          silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, bias);
+          if constexpr (kRab) load_bias<3>(bias, rab_row, rel0, rab_max);
           ptx::tmem_ld32(taddr_s + 96, ra);
           ptx::tmem_ld_wait(ra);
-          silu_chunk<3, kRab>(ra, taddr_s, half_alpha, full, lim, self, rab_row, rel0, rab_max);
+          silu_chunk<3, kRab>(ra, taddr_s, half_alpha, full, lim, self, bias);
           ptx::tmem_st_wait();
           ptx::tc_fence_before();
           __syncwarp();
