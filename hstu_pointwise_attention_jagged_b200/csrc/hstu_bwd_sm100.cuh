@@ -108,28 +108,38 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_
                                           uint32_t t_ds, float half_alpha, float ds_scale, bool full, int lo, int hi,
                                           int self) {
   uint32_t pk_p[16], pk_ds[16];
+  // Columns are taken in pairs on the two-wide FMA pipe; every lane rounds exactly as the scalar
+  // form h = s alpha/2, a = 1 + t, w = (h - h t) + 1, ds = ((dp ds_scale) a) w, p = h a would.
+  const uint64_t ha2 = ptx::f32x2(half_alpha, half_alpha);
+  const uint64_t sc2 = ptx::f32x2(ds_scale, ds_scale);
+  const uint64_t one2 = ptx::f32x2(1.0f, 1.0f);
+  const uint64_t neg2 = ptx::f32x2(-1.0f, -1.0f);
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
-    float p2[2], d2[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int c = 2 * e + u;
-      const float h = __uint_as_float(s[c]) * half_alpha;
-      const float t = ptx::tanh_approx(h);
-      const float a = 1.0f + t;
-      const float w = fmaf(-h, t, h) + 1.0f;
-      float ds = __uint_as_float(dp[c]) * ds_scale * a * w;
-      float p = h * a;
-      if (!full) {
-        const bool vis = (c >= lo && c < hi) || c == self;
-        ds = vis ? ds : 0.0f;
-        p = vis ? p : 0.0f;
+    const int c = 2 * e;
+    const uint64_t h2 = ptx::mul_f32x2(ptx::f32x2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), ha2);
+    float h0, h1;
+    ptx::f32x2_split(h2, h0, h1);
+    const uint64_t t2 = ptx::f32x2(ptx::tanh_approx(h0), ptx::tanh_approx(h1));
+    const uint64_t a2 = ptx::fma_f32x2(t2, one2, one2);
+    const uint64_t w2 = ptx::fma_f32x2(ptx::fma_f32x2(ptx::mul_f32x2(h2, neg2), t2, h2), one2, one2);
+    const uint64_t d2 = ptx::mul_f32x2(
+        ptx::mul_f32x2(ptx::mul_f32x2(ptx::f32x2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), sc2), a2), w2);
+    float ds0, ds1, p0, p1;
+    ptx::f32x2_split(d2, ds0, ds1);
+    if constexpr (!kDQ) ptx::f32x2_split(ptx::mul_f32x2(h2, a2), p0, p1);
+    if (!full) {
+      const bool v0 = (c >= lo && c < hi) || c == self;
+      const bool v1 = (c + 1 >= lo && c + 1 < hi) || c + 1 == self;
+      ds0 = v0 ? ds0 : 0.0f;
+      ds1 = v1 ? ds1 : 0.0f;
+      if constexpr (!kDQ) {
+        p0 = v0 ? p0 : 0.0f;
+        p1 = v1 ? p1 : 0.0f;
       }
-      p2[u] = p;
-      d2[u] = ds;
     }
-    pk_ds[e] = pack_bf16x2(d2[0], d2[1]);
-    if constexpr (!kDQ) pk_p[e] = pack_bf16x2(p2[0], p2[1]);
+    pk_ds[e] = pack_bf16x2(ds0, ds1);
+    if constexpr (!kDQ) pk_p[e] = pack_bf16x2(p0, p1);
   }
   ptx::tmem_st16(t_ds, pk_ds);
   if constexpr (!kDQ) ptx::tmem_st16(t_p, pk_p);
