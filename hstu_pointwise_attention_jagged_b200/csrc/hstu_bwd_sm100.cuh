@@ -72,7 +72,9 @@ template <int kStages>
 struct BwdCtl {
   uint64_t fix_full, fix_empty;
   uint64_t ring_full[kStages], ring_empty[kStages];
-  uint64_t s_full, p_full, o_full, o_empty;
+  // s_full / dp_full: the score MMAs of a tile committed; p_full: the elementwise warps are done with
+  // S (dK/dV: P written; dQ: S read); ds_full: dS written.
+  uint64_t s_full, dp_full, p_full, ds_full, o_full, o_empty;
   uint64_t sched_full[2], sched_empty[2];
   uint64_t drain;
   // work slot: valid, h, row0 (first token row of the user), fixed tile, L, U, e1, s2, e2
@@ -100,18 +102,16 @@ __device__ __forceinline__ BwdWork read_bwd_slot(const volatile int32_t* s) {
   return w;
 }
 
-// 32 score columns of this thread's row: S and dP chunks in registers -> dS (and, for dK/dV, P)
-// packed as bf16 pairs into 16 TMEM columns each.  The visible columns are [lo, hi) plus `self`
-// (relative to the chunk's first column), everything else is an exact zero.
+// First half of the elementwise step, 32 score columns of this thread's row.  From S it forms the
+// SiLU factor m = (1 + t)(1 + h - h t) of every column, kept in registers for the second half, and
+// (dK/dV) P = h (1 + t), packed as bf16 pairs into 16 TMEM columns.  The visible columns are
+// [lo, hi) plus `self` (relative to the chunk's first column); P is an exact zero elsewhere.
+// Columns go in pairs on the two-wide FMA pipe.
 template <bool kDQ>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], uint32_t t_p,
-                                          uint32_t t_ds, float half_alpha, float ds_scale, bool full, int lo, int hi,
-                                          int self) {
-  uint32_t pk_p[16], pk_ds[16];
-  // Columns are taken in pairs on the two-wide FMA pipe; every lane rounds exactly as the scalar
-  // form h = s alpha/2, a = 1 + t, w = (h - h t) + 1, ds = ((dp ds_scale) a) w, p = h a would.
+__device__ __forceinline__ void bwd_scores(const uint32_t (&s)[32], float (&m)[32], uint32_t t_p, float half_alpha,
+                                           bool full, int lo, int hi, int self) {
+  uint32_t pk_p[16];
   const uint64_t ha2 = ptx::f32x2(half_alpha, half_alpha);
-  const uint64_t sc2 = ptx::f32x2(ds_scale, ds_scale);
   const uint64_t one2 = ptx::f32x2(1.0f, 1.0f);
   const uint64_t neg2 = ptx::f32x2(-1.0f, -1.0f);
 #pragma unroll
@@ -121,28 +121,42 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_
     float h0, h1;
     ptx::f32x2_split(h2, h0, h1);
     const uint64_t t2 = ptx::f32x2(ptx::tanh_approx(h0), ptx::tanh_approx(h1));
-    const uint64_t a2 = ptx::fma_f32x2(t2, one2, one2);
-    const uint64_t w2 = ptx::fma_f32x2(ptx::fma_f32x2(ptx::mul_f32x2(h2, neg2), t2, h2), one2, one2);
-    const uint64_t d2 = ptx::mul_f32x2(
-        ptx::mul_f32x2(ptx::mul_f32x2(ptx::f32x2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), sc2), a2), w2);
-    float ds0, ds1, p0, p1;
-    ptx::f32x2_split(d2, ds0, ds1);
-    if constexpr (!kDQ) ptx::f32x2_split(ptx::mul_f32x2(h2, a2), p0, p1);
-    if (!full) {
-      const bool v0 = (c >= lo && c < hi) || c == self;
-      const bool v1 = (c + 1 >= lo && c + 1 < hi) || c + 1 == self;
-      ds0 = v0 ? ds0 : 0.0f;
-      ds1 = v1 ? ds1 : 0.0f;
-      if constexpr (!kDQ) {
-        p0 = v0 ? p0 : 0.0f;
-        p1 = v1 ? p1 : 0.0f;
+    const uint64_t a2 = ptx::fma_f32x2(t2, one2, one2);                                          // 1 + t
+    const uint64_t w2 = ptx::fma_f32x2(ptx::fma_f32x2(ptx::mul_f32x2(h2, neg2), t2, h2), one2, one2);  // 1 + h - h t
+    ptx::f32x2_split(ptx::mul_f32x2(a2, w2), m[c], m[c + 1]);
+    if constexpr (!kDQ) {
+      float p0, p1;
+      ptx::f32x2_split(ptx::mul_f32x2(h2, a2), p0, p1);
+      if (!full) {
+        p0 = ((c >= lo && c < hi) || c == self) ? p0 : 0.0f;
+        p1 = ((c + 1 >= lo && c + 1 < hi) || c + 1 == self) ? p1 : 0.0f;
       }
+      pk_p[e] = pack_bf16x2(p0, p1);
     }
-    pk_ds[e] = pack_bf16x2(ds0, ds1);
-    if constexpr (!kDQ) pk_p[e] = pack_bf16x2(p0, p1);
   }
-  ptx::tmem_st16(t_ds, pk_ds);
   if constexpr (!kDQ) ptx::tmem_st16(t_p, pk_p);
+}
+
+// Second half: dS = (dP ds_scale) m, an exact zero outside the visible columns, packed as bf16
+// pairs into 16 TMEM columns.
+__device__ __forceinline__ void bwd_grads(const uint32_t (&dp)[32], const float (&m)[32], uint32_t t_ds,
+                                          float ds_scale, bool full, int lo, int hi, int self) {
+  uint32_t pk[16];
+  const uint64_t sc2 = ptx::f32x2(ds_scale, ds_scale);
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int c = 2 * e;
+    float d0, d1;
+    ptx::f32x2_split(ptx::mul_f32x2(ptx::mul_f32x2(ptx::f32x2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), sc2),
+                                    ptx::f32x2(m[c], m[c + 1])),
+                     d0, d1);
+    if (!full) {
+      d0 = ((c >= lo && c < hi) || c == self) ? d0 : 0.0f;
+      d1 = ((c + 1 >= lo && c + 1 < hi) || c + 1 == self) ? d1 : 0.0f;
+    }
+    pk[e] = pack_bf16x2(d0, d1);
+  }
+  ptx::tmem_st16(t_ds, pk);
 }
 
 template <int D, bool kDQ>
@@ -172,7 +186,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ptx::mbar_init(bar(ctl->ring_empty[s]), 1);
     }
     ptx::mbar_init(bar(ctl->s_full), 1);
+    ptx::mbar_init(bar(ctl->dp_full), 1);
     ptx::mbar_init(bar(ctl->p_full), 8);
+    ptx::mbar_init(bar(ctl->ds_full), 8);
     ptx::mbar_init(bar(ctl->o_full), 1);
     ptx::mbar_init(bar(ctl->o_empty), 8);
     for (int i = 0; i < 2; ++i) {
@@ -284,27 +300,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t dringmn = ptx::smem_desc(sRing, T::kBlockBytes, 8 * T::kRowBytes, T::kSwizzle);  // MN-major B
     int slot = 0;
     uint32_t sched_full_par[2] = {0u, 0u};
-    uint32_t fix_full_par = 0u, p_full_par = 0u, o_empty_par = 1u;
+    uint32_t fix_full_par = 0u, p_full_par = 0u, ds_full_par = 0u, o_empty_par = 1u;
     int stage = 0;
     uint32_t ring_phase = 0;
     bool ok = true;
-    // Accumulating MMAs of streamed tile `st` (ring stage `sst`), whose P / dS are in TMEM.
-    auto accumulate = [&](int sst, bool first) {
-      const uint64_t base_mn = dringmn + ((sst * 2 * T::kTileBytes) >> 4);
+    // Score MMAs of the streamed tile in ring stage `sst`: which = 0 gives S (fixed[0] x
+    // streamed[0]^T), which = 1 gives dP (fixed[1] x streamed[1]^T).
+    auto scores = [&](int sst, int which) {
+      const uint64_t dst = dring + ((sst * 2 * T::kTileBytes + which * T::kTileBytes) >> 4);
+      const uint64_t dfx = dfix + ((which * T::kTileBytes) >> 4);
+      const uint32_t col = which ? Cfg::kColDP : Cfg::kColS;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t off = (ks / T::kKStepsPerBlock) * T::kBlockBytes + (ks % T::kKStepsPerBlock) * 32;
+        ptx::mma_ss_lead(lead, tmem + col, dfx + (off >> 4), dst + (off >> 4), Cfg::kIdescScore, ks > 0 ? 1u : 0u);
+      }
+    };
+    // acc += A B with A (bf16 P or dS) read from TMEM at column a_col and B the streamed tile `which`
+    // of ring stage `sst` (MN-major); `first` starts the accumulator afresh.
+    auto accum = [&](int sst, uint32_t acc_col, uint32_t a_col, int which, bool first) {
+      const uint64_t dmn = dringmn + ((sst * 2 * T::kTileBytes + which * T::kTileBytes) >> 4);
 #pragma unroll
       for (int ks = 0; ks < kTileRows / 16; ++ks) {
         const uint32_t acol = 64 * (ks >> 2) + 8 * (ks & 3);
-        const uint32_t acc = (first && ks == 0) ? 0u : 1u;
-        const uint64_t boff = (ks * 16 * T::kRowBytes) >> 4;
-        if constexpr (kDQ) {
-          // dQ += dS K: dS from the dP columns, K = streamed tile 0.
-          ptx::mma_ts_lead(lead, tmem + Cfg::kColA0, tmem + Cfg::kColDP + acol, base_mn + boff, Cfg::kIdescAcc, acc);
-        } else {
-          // dV += P^T dO (dO = streamed tile 1), dK += dS^T Q (Q = streamed tile 0).
-          ptx::mma_ts_lead(lead, tmem + Cfg::kColA0, tmem + Cfg::kColS + acol,
-                           base_mn + ((T::kTileBytes) >> 4) + boff, Cfg::kIdescAcc, acc);
-          ptx::mma_ts_lead(lead, tmem + Cfg::kColA1, tmem + Cfg::kColDP + acol, base_mn + boff, Cfg::kIdescAcc, acc);
-        }
+        ptx::mma_ts_lead(lead, tmem + acc_col, tmem + a_col + acol, dmn + ((ks * 16 * T::kRowBytes) >> 4),
+                         Cfg::kIdescAcc, (first && ks == 0) ? 0u : 1u);
+      }
+    };
+    auto next_stage = [&]() {
+      if (++stage == Cfg::kStages) {
+        stage = 0;
+        ring_phase ^= 1u;
       }
     };
     while (ok) {
@@ -318,42 +344,61 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int n = tile_count(w.r);
       if (!wait_all(bar(ctl->fix_full), fix_full_par)) break;
       fix_full_par ^= 1u;
-      ptx::tc_fence_after();
-      int prev_stage = 0;
-      for (int i = 0; i <= n && ok; ++i) {
-        if (i > 0) {
-          // The previous tile's P / dS are in TMEM: accumulate, then free its ring stage.
-          ok = wait_all(bar(ctl->p_full), p_full_par) && (i > 1 || wait_all(bar(ctl->o_empty), o_empty_par));
-          if (!ok) break;
-          p_full_par ^= 1u;
-          if (i == 1) o_empty_par ^= 1u;
+      // Tile 0's scores.
+      int cur = stage;
+      if (n > 0) {
+        if (!wait_all(bar(ctl->ring_full[stage]), ring_phase)) break;
+        next_stage();
+        ptx::tc_fence_after();
+        scores(cur, 0);
+        ptx::mma_commit_lead(lead, bar(ctl->s_full));
+        scores(cur, 1);
+        ptx::mma_commit_lead(lead, bar(ctl->dp_full));
+      }
+      // Tile i's gradient MMAs wait for its elementwise halves; tile i+1's score MMAs fill the gaps.
+      //   dK/dV:  dV(i) [P_i]  S(i+1)  dK(i) [dS_i]  dP(i+1)
+      //   dQ:     S(i+1) [S_i read]  dQ(i) [dS_i]  dP(i+1)
+      // Every overwrite of a TMEM buffer is issued after the MMA that last reads it (tcgen05 MMAs of
+      // one thread run in order), and after the elementwise warps have released it.
+      for (int i = 0; i < n && ok; ++i) {
+        const bool more = i + 1 < n;
+        const int nxt = stage;
+        const uint32_t nph = ring_phase;
+        if (more) next_stage();
+        ok = wait_all(bar(ctl->p_full), p_full_par);
+        if (!ok) break;
+        p_full_par ^= 1u;
+        if constexpr (!kDQ) {
+          if (i == 0) {
+            if (!wait_all(bar(ctl->o_empty), o_empty_par)) { ok = false; break; }
+            o_empty_par ^= 1u;
+          }
           ptx::tc_fence_after();
-          accumulate(prev_stage, i == 1);
-          ptx::mma_commit_lead(lead, bar(ctl->ring_empty[prev_stage]));
+          accum(cur, Cfg::kColA0, Cfg::kColS, 1, i == 0);  // dV += P^T dO
         }
-        if (i < n) {
-          if (!wait_all(bar(ctl->ring_full[stage]), ring_phase)) {
-            ok = false;
-            break;
-          }
+        if (more) {
+          if (!wait_all(bar(ctl->ring_full[nxt]), nph)) { ok = false; break; }
           ptx::tc_fence_after();
-          const uint64_t ds0 = dring + ((stage * 2 * T::kTileBytes) >> 4);
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks / T::kKStepsPerBlock) * T::kBlockBytes + (ks % T::kKStepsPerBlock) * 32;
-            // scores: fixed[0] x streamed[0]^T -> S;  fixed[1] x streamed[1]^T -> dP
-            ptx::mma_ss_lead(lead, tmem + Cfg::kColS, dfix + (off >> 4), ds0 + (off >> 4), Cfg::kIdescScore,
-                             ks > 0 ? 1u : 0u);
-            ptx::mma_ss_lead(lead, tmem + Cfg::kColDP, dfix + ((T::kTileBytes + off) >> 4),
-                             ds0 + ((T::kTileBytes + off) >> 4), Cfg::kIdescScore, ks > 0 ? 1u : 0u);
-          }
+          scores(nxt, 0);
           ptx::mma_commit_lead(lead, bar(ctl->s_full));
-          prev_stage = stage;
-          if (++stage == Cfg::kStages) {
-            stage = 0;
-            ring_phase ^= 1u;
+        }
+        if (!wait_all(bar(ctl->ds_full), ds_full_par)) { ok = false; break; }
+        ds_full_par ^= 1u;
+        if constexpr (kDQ) {
+          if (i == 0) {
+            if (!wait_all(bar(ctl->o_empty), o_empty_par)) { ok = false; break; }
+            o_empty_par ^= 1u;
           }
         }
+        ptx::tc_fence_after();
+        if constexpr (kDQ) accum(cur, Cfg::kColA0, Cfg::kColDP, 0, i == 0);  // dQ += dS K
+        else accum(cur, Cfg::kColA1, Cfg::kColDP, 0, i == 0);                // dK += dS^T Q
+        ptx::mma_commit_lead(lead, bar(ctl->ring_empty[cur]));  // tile i's streamed pair is done
+        if (more) {
+          scores(nxt, 1);
+          ptx::mma_commit_lead(lead, bar(ctl->dp_full));
+        }
+        cur = nxt;
       }
       if (!ok) break;
       ptx::mma_commit_lead(lead, bar(ctl->fix_empty));  // fixed pair free after the item's last MMA
@@ -372,7 +417,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_dp = tmem + lane_off + Cfg::kColDP + 64 * ch;
     int slot = 0;
     uint32_t sched_full_par[2] = {0u, 0u};
-    uint32_t s_full_par = 0u, o_full_par = 0u;
+    uint32_t s_full_par = 0u, dp_full_par = 0u, o_full_par = 0u;
     bool ok = true;
     while (ok) {
       ok = __all_sync(0xffffffffu, wait_bounded(bar(ctl->sched_full[slot]), sched_full_par[slot], abort_flag, p.err));
@@ -408,20 +453,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           self = -1;
           full = (lo <= 0) && (hi >= 64);
         }
+        // First half: S -> the SiLU factors (registers) and, for dK/dV, P over S.  Then S is released.
+        float m[2][32];
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-          uint32_t rs[32], rd[32];
+          uint32_t rs[32];
           ptx::tmem_ld32(t_s + 32 * k, rs);
-          ptx::tmem_ld32(t_dp + 32 * k, rd);
           ptx::tmem_ld_wait(rs);
+          bwd_scores<kDQ>(rs, m[k], t_s + 16 * k, p.half_alpha, full, lo - 32 * k, hi - 32 * k, self - 32 * k);
+        }
+        if constexpr (!kDQ) ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(ctl->p_full));
+        // Second half: dP -> dS over dP.
+        ok = __all_sync(0xffffffffu, wait_bounded(bar(ctl->dp_full), dp_full_par, abort_flag, p.err));
+        if (!ok) break;
+        dp_full_par ^= 1u;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          uint32_t rd[32];
+          ptx::tmem_ld32(t_dp + 32 * k, rd);
           ptx::tmem_ld_wait(rd);
-          bwd_chunk<kDQ>(rs, rd, t_s + 16 * k, t_dp + 16 * k, p.half_alpha, p.ds_scale, full, lo - 32 * k,
-                         hi - 32 * k, self - 32 * k);
+          bwd_grads(rd, m[k], t_dp + 16 * k, p.ds_scale, full, lo - 32 * k, hi - 32 * k, self - 32 * k);
         }
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(ctl->p_full));
+        if (lane == 0) ptx::mbar_arrive(bar(ctl->ds_full));
       }
       if (!ok) break;
       ok = __all_sync(0xffffffffu, wait_bounded(bar(ctl->o_full), o_full_par, abort_flag, p.err));
