@@ -98,6 +98,13 @@ def test_single_long_user():
     assert torch.isfinite(got_all.float()).all()
 
 
+def test_long_users_head32():
+    """d = 32 with long users: sub-items of up to 24 key tiles, so the 10-slot K/V ring and the
+    rotating score-commit barriers wrap many times at this head size; every row compared."""
+    w = workloads.make_custom("long32", [2600, 1900, 7], [500, 260, 2], 2, 32, 1 / math.sqrt(32), 3100.0, seed=80)
+    _full_compare(w, "long users d=32")
+
+
 @pytest.mark.parametrize("name", ["dlrmv3", "jagged", "long_history"])
 def test_full_size_sampled(name):
     """Full-size named workloads, one launch as the bench times it; sampled rows vs the oracle."""
