@@ -140,21 +140,21 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 // Plan layout (documented in include/hstu_attn.h):
 //   int32 header[4] = {work counter, num_items, done counter, 0}
 //   int32 q_start[B], padded to 16 bytes
-//   int32 pair_start[B+1], padded to 16 bytes
-//   int4  items[capacity] = {b, pair, h, cost}, capacity = H * (total_q / 256 + B)
+//   int32 block_start[B+1], padded to 16 bytes
+//   int4  items[capacity] = {b, block, h, cost}, capacity = H * (total_q / 128 + B)
 struct Plan {
   int32_t* counter;
   int32_t* num_items;
   int32_t* done;
   int32_t* q_start;
-  int32_t* pair_start;
+  int32_t* block_start;
   int4* items;
 };
 
 size_t pad16(size_t n_ints) { return ((n_ints * 4 + 15) / 16) * 16; }
 
 int64_t capacity(int32_t B, int32_t H, int32_t total_q) {
-  return static_cast<int64_t>(H) * (total_q / kPairRows + B);
+  return static_cast<int64_t>(H) * (total_q / kItemRows + B);
 }
 
 int64_t plan_bytes(int32_t B, int32_t H, int32_t total_q) {
@@ -168,13 +168,13 @@ Plan carve(void* base, int32_t B) {
   w.num_items = reinterpret_cast<int32_t*>(p + 4);
   w.done = reinterpret_cast<int32_t*>(p + 8);
   w.q_start = reinterpret_cast<int32_t*>(p + 16);
-  w.pair_start = reinterpret_cast<int32_t*>(p + 16 + pad16(B));
+  w.block_start = reinterpret_cast<int32_t*>(p + 16 + pad16(B));
   w.items = reinterpret_cast<int4*>(p + 16 + pad16(B) + pad16(static_cast<size_t>(B) + 1));
   return w;
 }
 
 int cost_bins(int32_t max_seq_len) {
-  // A 256-row item computes at most 2 * (ceil(L/128) + 1) score tiles.
+  // A 128-row item computes at most ceil(L/128) + 1 score tiles; the bins leave twice that room.
   int64_t n = 2 * (static_cast<int64_t>(max_seq_len) / kTileRows + 3) + 1;
   return static_cast<int>(n < kMaxCostBins ? n : kMaxCostBins);
 }
@@ -217,7 +217,7 @@ cudaError_t launch_plan(const int32_t* seq_offsets, const int32_t* num_targets, 
   a.nbins = cost_bins(max_seq_len);
   a.max_items = static_cast<int32_t>(capacity(B, H, total_q));
   a.q_start = w.q_start;
-  a.pair_start = w.pair_start;
+  a.block_start = w.block_start;
   a.items = w.items;
   a.num_items = w.num_items;
   a.work_counter = w.counter;

@@ -1,12 +1,11 @@
 // hstu_fwd_sm100.cuh — fused forward kernel of jagged target-aware HSTU pointwise attention for
 // sm_100a:  out = Mask(SiLU(alpha * Q K^T)) V / N   (DLRMv3 review, section "model selection").
 //
-// One persistent CTA per SM pulls work items (user b, head h, up to 256 query rows) from a cost-
-// ordered list through an atomic counter.  Each item is worked as one or two 128-row sub-items
-// (query tiles); every role walks the same global sequence of score tiles g = 0, 1, 2, ... over
-// the CTA's sub-items and their visible key tiles.
+// One persistent CTA per SM pulls work items (user b, head h, one tile of up to 128 query rows)
+// from a cost-ordered list through an atomic counter.  Every role walks the same global sequence
+// of score tiles g = 0, 1, 2, ... over the CTA's query tiles and their visible key tiles.
 //
-//   warp 8       producer: fetches the next item, TMA-loads each sub-item's Q into one of two
+//   warp 8       producer: fetches the next item, TMA-loads each query tile's Q into one of two
 //                buffers and the K and V tiles into a ring of shared-memory slots, in the order
 //                the tensor core consumes them: K_0 K_1 K_2 V_0 K_3 V_1 K_4 ... (V_{g-3}, K_g).
 //   warp 9       MMA issuer (lane 0 issues every tcgen05 instruction).  Group g is
@@ -16,16 +15,16 @@
 //   warps 0-3,   SiLU warpgroups; warpgroup g mod 2 takes tile g: TMEM -> registers, p = mask ?
 //   warps 4-7    silu(alpha*s) : 0 with silu(x) = h + h*tanh(h), h = x/2 (one MUFU op per score),
 //                packed to bf16 and written back over S_g in TMEM.
-//   warps 10-13  epilogue: after a sub-item's last P.V, O * (1/N) -> bf16 -> row-predicated
+//   warps 10-13  epilogue: after a query tile's last P.V, O * (1/N) -> bf16 -> row-predicated
 //                global stores.  O is released as soon as it is in registers, so the next
-//                sub-item's first P.V waits only for the TMEM reads.
+//                query tile's first P.V waits only for the TMEM reads.
 //
 // TMEM (512 columns x 128 lanes of fp32): O [0, D), score buffer b at [128 + 128 b, 256 + 128 b)
 // for b = 0, 1, 2.  P_g (bf16 pairs) overwrites the first 64 columns of its score buffer; the
 // next S MMA into that buffer is issued after the P.V that reads it, and tcgen05 MMAs from one
 // thread execute in order.
 //
-// Each group has one ready barrier: the producer's copies for it (Q on a sub-item's first tile,
+// Each group has one ready barrier: the producer's copies for it (Q with a query tile's first key tile,
 // V_{g-3}, K_g) complete their bytes on it and the four SiLU warps that wrote P_{g-3} arrive on it,
 // so the MMA warp makes one wait per group.  A ring slot is reused once the group that consumed
 // its previous tile has completed; the score commit of group G covers every MMA issued before it,
@@ -258,12 +257,6 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t tad
 // whole ring.)
 __device__ __forceinline__ int group_of_load(int e) { return e < 3 ? e : (e + 3) >> 1; }
 
-// Rows of sub-item hh of a work item (query rows [128 hh, 128 hh + 128)); <= 0 if it has none.
-__device__ __forceinline__ int sub_rows(const Work& w, int hh) {
-  const int r = w.nrows - hh * kTileRows;
-  return r < kTileRows ? r : kTileRows;
-}
-
 template <int D, bool kRab>
 __global__ void __launch_bounds__(kNumThreads, 1)
     hstu_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -320,7 +313,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       const int M = *p.num_items;
       int slot = 0;
       uint32_t sched_empty_par = (1u << kSlots) - 1u;  // bit s: parity of slot s's next wait
-      int sub = 0;        // sub-items whose Q load was issued
+      int sub = 0;        // query tiles whose Q load was issued
       int j = 0;          // K/V loads issued
       int g = 0;          // score tiles (groups with an S) armed
       int armed_hi = 0;   // one past the highest group index armed
@@ -352,10 +345,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const int T = p.num_targets ? p.num_targets[b] : 0;
           const int c = p.cached_len ? p.cached_len[b] : 0;
           w.U = w.L - T;
-          w.q_row0 = p.q_start[b] + pair * kPairRows;
-          w.pos0 = c + pair * kPairRows;
-          const int rows = (w.L - c) - pair * kPairRows;
-          w.nrows = rows < kPairRows ? rows : kPairRows;
+          w.q_row0 = p.q_start[b] + pair * kItemRows;
+          w.pos0 = c + pair * kItemRows;
+          const int rows = (w.L - c) - pair * kItemRows;
+          w.nrows = rows < kItemRows ? rows : kItemRows;
         }
         if (!wait_bounded(bar(ctl->sched_empty[slot]), (sched_empty_par >> slot) & 1u, abort_flag, p.err,
                           p.wait_limit_ns)) {
@@ -370,11 +363,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         slot = (slot + 1) & (kSlots - 1);
         if (!w.valid) break;
 
-        for (int hh = 0; hh < 2 && ok; ++hh) {
-          const int nr = sub_rows(w, hh);
-          if (nr <= 0) break;
-          const int lo = hh * kTileRows;
-          const TileRange r = key_tiles(w.pos0 + lo, w.pos0 + lo + nr, w.U);
+        {
+          const TileRange r = key_tiles(w.pos0, w.pos0 + w.nrows, w.U);
           const int n = tile_count(r);
           const int qb = sub & 1;
           if (!wait_bounded(bar(ctl->q_empty[qb]), (uint32_t)(((sub >> 1) & 1) ^ 1), abort_flag, p.err,
@@ -384,7 +374,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           }
           for (int k = 0; k < n; ++k) {
             // Group g reads V_{g-3} (load j) and K_g (load j+1), or K_g alone for g < 3, and Q on
-            // a sub-item's first tile; all of them land on the group's ready barrier.
+            // a query tile's first tile; all of them land on the group's ready barrier.
             const bool has_v = g >= 3;
             if (!slot_free(j) || (has_v && !slot_free(j + 1))) { ok = false; break; }
             const int krow = w.kv_start + tile_at(r, k) * kTileRows;
@@ -393,7 +383,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             if (!has_v)  // no P.V in this group: stand in for the SiLU warps' arrivals
               for (int a = 0; a < 4; ++a) ptx::mbar_arrive(rb);
             if (k == 0) {
-              tma_tile(&tm_q, sQ + qb * Cfg::kTileBytes, rb, w.h * D, w.q_row0 + lo);
+              tma_tile(&tm_q, sQ + qb * Cfg::kTileBytes, rb, w.h * D, w.q_row0);
               ++sub;
             }
             if (has_v) {
@@ -460,11 +450,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     int r8 = 0;              // g mod kGroupBars: ready barrier of group g
     uint32_t rpar = 0u;      // parity of that barrier's phase for group g
     uint32_t o_empty_par = 1u;
-    // Tiles g-3, g-2, g-1: bit 0 = first tile of its sub-item, bit 1 = last tile of its sub-item.
+    // Tiles g-3, g-2, g-1: bit 0 = first tile of its query tile, bit 1 = last tile of its query tile.
     uint32_t f0 = 0, f1 = 0, f2 = 0;
     bool ok = true;
     // O += P V for a tile whose P is in score buffer pb and whose V is in ring slot vs (its group's
-    // ready barrier already waited).  A sub-item's first tile starts O afresh once the epilogue
+    // ready barrier already waited).  A query tile's first tile starts O afresh once the epilogue
     // has read the previous O; its last one commits O to the epilogue.
     auto issue_pv = [&](uint32_t pb, int vs, uint32_t flags) {
       if (flags & 1u) {
@@ -494,11 +484,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       slot = (slot + 1) & (kSlots - 1);
       if (!w.valid) break;
 
-      for (int hh = 0; hh < 2 && ok; ++hh) {
-        const int nr = sub_rows(w, hh);
-        if (nr <= 0) break;
-        const int lo = hh * kTileRows;
-        const TileRange r = key_tiles(w.pos0 + lo, w.pos0 + lo + nr, w.U);
+      {
+        const TileRange r = key_tiles(w.pos0, w.pos0 + w.nrows, w.U);
         const int n = tile_count(r);
         const int qb = sub & 1;
         const uint64_t dq = dq0 + ((qb * Cfg::kTileBytes) >> 4);
@@ -571,11 +558,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
       const float* rab_row = kRab ? p.rab + (size_t)w.h * p.rab_len : nullptr;
       const int rab_max = kRab ? p.rab_len - 1 : 0;
-      for (int hh = 0; hh < 2 && ok; ++hh) {
-        const int nr = sub_rows(w, hh);
-        if (nr <= 0) break;
-        const int p0 = w.pos0 + hh * kTileRows;
-        const TileRange r = key_tiles(p0, p0 + nr, w.U);
+      {
+        const int p0 = w.pos0;
+        const TileRange r = key_tiles(p0, p0 + w.nrows, w.U);
         const int n = tile_count(r);
         const int i_pos = p0 + row;                           // this thread's query position
         const int lim_abs = (i_pos < w.U) ? i_pos + 1 : w.U;  // keys [0, lim_abs) visible, plus self
@@ -644,15 +629,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       slot = (slot + 1) & (kSlots - 1);
       if (!w.valid) break;
 
-      for (int hh = 0; hh < 2 && ok; ++hh) {
-        const int nr = sub_rows(w, hh);
-        if (nr <= 0) break;
+      {
+        const int nr = w.nrows;
         ok = wait_bounded(bar(ctl->o_full), o_full_par, abort_flag, p.err, p.wait_limit_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         o_full_par ^= 1u;
         ptx::tc_fence_after();
-        // O * (1/N) -> bf16 pairs in registers; O is then released to the next sub-item's P.V.
+        // O * (1/N) -> bf16 pairs in registers; O is then released to the next query tile's P.V.
         uint32_t a[D / 2];
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -667,7 +651,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(ctl->o_empty));
         if (row < nr) {
-          const size_t orow = (size_t)(w.q_row0 + hh * kTileRows + row);
+          const size_t orow = (size_t)(w.q_row0 + row);
           const size_t col = (size_t)w.h * D;
           uint4* dst = reinterpret_cast<uint4*>(p.out + orow * p.out_ld + col);
 #pragma unroll

@@ -17,7 +17,7 @@
 namespace hstu {
 
 constexpr int kTileRows = 128;  // query rows per half / keys per key tile
-constexpr int kPairRows = 256;  // query rows per work item (two 128-row halves)
+constexpr int kItemRows = 128;  // query rows per work item: one query tile
 
 __host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
@@ -55,17 +55,10 @@ __host__ __device__ __forceinline__ bool tile_in(const TileRange& r, int t) {
   return t < r.e1 || (t >= r.s2 && t < r.e2);
 }
 
-// Score tiles computed by one work item: query rows [256*pair, 256*pair + nrows) at positions
-// pos0.. of a segment with U history tokens, split into two 128-row halves.
-__host__ __device__ __forceinline__ int pair_cost(int pos0, int nrows, int U) {
-  int c = 0;
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int lo = hh * kTileRows;
-    const int hi = (nrows < lo + kTileRows) ? nrows : lo + kTileRows;
-    if (hi > lo) c += tile_count(key_tiles(pos0 + lo, pos0 + hi, U));
-  }
-  return c;
+// Score tiles computed by one work item: query rows [128*blk, 128*blk + nrows) at positions
+// pos0.. of a segment with U history tokens.
+__host__ __device__ __forceinline__ int item_cost(int pos0, int nrows, int U) {
+  return nrows > 0 ? tile_count(key_tiles(pos0, pos0 + nrows, U)) : 0;
 }
 
 constexpr unsigned kErrBadOffsets = 1u;
@@ -81,7 +74,7 @@ struct SchedArgs {
   const int32_t* cached_len;   // [B] or null
   int32_t B, H, total_kv, total_q, max_seq_len, nbins, max_items;
   int32_t* q_start;       // [B] out: first query row of each user, -1 if the user is skipped
-  int32_t* pair_start;    // [B+1] out: index of each user's first 256-row block among all blocks
+  int32_t* block_start;    // [B+1] out: index of each user's first 128-row block among all blocks
   int4* items;            // [max_items] out: {b, pair, h, cost}, non-increasing cost
   int32_t* num_items;     // [1] out
   int32_t* work_counter;  // [1] out: reset to 0 for the attention kernel's dynamic scheduler
@@ -160,20 +153,20 @@ __device__ __forceinline__ long long block_inclusive_scan(long long v, long long
   return v;
 }
 
-// User owning block g: the last b with pair_start[b] <= g (users without blocks share a start).
-// pair_start may live in shared or global memory.
-__device__ __forceinline__ int owner_of(const int32_t* pair_start, int B, int g) {
-  int lo = 0, hi = B;  // pair_start[lo] <= g < pair_start[hi]
+// User owning block g: the last b with block_start[b] <= g (users without blocks share a start).
+// block_start may live in shared or global memory.
+__device__ __forceinline__ int owner_of(const int32_t* block_start, int B, int g) {
+  int lo = 0, hi = B;  // block_start[lo] <= g < block_start[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (pair_start[mid] <= g) lo = mid; else hi = mid;
+    if (block_start[mid] <= g) lo = mid; else hi = mid;
   }
   return lo;
 }
 
 // One CTA of kSchedThreads threads.  Validates every user, assigns query-row starts, and writes
 // the work items sorted by non-increasing cost (counting sort over cost bins; ties in any order).
-// The per-block passes run one thread per (user, 256-row block).
+// The per-block passes run one thread per (user, 128-row block).
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs a) {
   // A dependent attention kernel may start its prologue now; it waits for this grid's writes
   // (griddepcontrol.wait) before it reads anything in global memory.
@@ -200,7 +193,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
   // and the block starts.  Lengths are taken in 64 bits, so that corrupt offsets cannot wrap.
   for (int base = 0; base < a.B; base += kSchedThreads) {
     const int b = base + tid;
-    long long nq = 0, npairs = 0;  // rows in the layout; 256-row blocks to compute
+    long long nq = 0, nblocks = 0;  // rows in the layout; 128-row blocks to compute
     bool ok = false;
     int L = 0, T = 0, c = 0;
     if (b < a.B) {
@@ -219,19 +212,19 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
       const long long cc = c < 0 ? 0 : c;
       nq = L64 > cc ? L64 - cc : 0;
       if (nq > (long long)a.total_q + 1) nq = (long long)a.total_q + 1;
-      npairs = ok ? cdiv(L - c, kPairRows) : 0;
+      nblocks = ok ? cdiv(L - c, kItemRows) : 0;
     }
-    long long incl_q = nq, incl_p = npairs, tot_q, tot_p;
+    long long incl_q = nq, incl_p = nblocks, tot_q, tot_p;
     block_inclusive_scan2(incl_q, incl_p, scan_scratch, tot_q, tot_p);
     const long long start_q = carry_q + incl_q - nq;
-    const long long start_p = carry_p + incl_p - npairs;
+    const long long start_p = carry_p + incl_p - nblocks;
     if (b < a.B) {
       if (ok && (start_q < 0 || start_q + nq > a.total_q)) {
         ok = false;
         atomicOr(a.err, kErrBadOffsets);
       }
       a.q_start[b] = ok ? (int)start_q : -1;
-      a.pair_start[b] = (int)start_p;
+      a.block_start[b] = (int)start_p;
       if (cached) {
         s_L[b] = L;
         s_U[b] = L - T;
@@ -247,28 +240,28 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
     }
     __syncthreads();
   }
-  const int npairs_total = (int)carry_p;
+  const int nblocks_total = (int)carry_p;
   if (tid == 0) {
-    a.pair_start[a.B] = npairs_total;
-    if (cached) s_ps[a.B] = npairs_total;
+    a.block_start[a.B] = nblocks_total;
+    if (cached) s_ps[a.B] = nblocks_total;
     if (carry_q != a.total_q) atomicOr(a.err, kErrBadOffsets);
   }
   __syncthreads();
   // Cost of block g (and its user), from shared memory when cached.
   auto block_of = [&](int g, int& b, int& pr, int& cost) {
-    b = owner_of(cached ? s_ps : a.pair_start, a.B, g);
+    b = owner_of(cached ? s_ps : a.block_start, a.B, g);
     if ((cached ? s_q[b] : a.q_start[b]) < 0) return false;
     const int L = cached ? s_L[b] : a.seq_offsets[b + 1] - a.seq_offsets[b];
     const int U = cached ? s_U[b] : L - (a.num_targets ? a.num_targets[b] : 0);
     const int c = cached ? s_c[b] : (a.cached_len ? a.cached_len[b] : 0);
-    pr = g - (cached ? s_ps[b] : a.pair_start[b]);
-    const int rows = (L - c) - pr * kPairRows;
-    cost = pair_cost(c + pr * kPairRows, rows < kPairRows ? rows : kPairRows, U);
+    pr = g - (cached ? s_ps[b] : a.block_start[b]);
+    const int rows = (L - c) - pr * kItemRows;
+    cost = item_cost(c + pr * kItemRows, rows < kItemRows ? rows : kItemRows, U);
     return true;
   };
 
   // Pass 2: cost histogram, one thread per block.
-  for (int g = tid; g < npairs_total; g += kSchedThreads) {
+  for (int g = tid; g < nblocks_total; g += kSchedThreads) {
     int b, pr, cost;
     if (!block_of(g, b, pr, cost)) continue;
     atomicAdd(&hist[cost < nbins ? cost : nbins - 1], a.H);
@@ -302,7 +295,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
   }
 
   // Pass 4: scatter the items into their bins, one thread per block.
-  for (int g = tid; g < npairs_total; g += kSchedThreads) {
+  for (int g = tid; g < nblocks_total; g += kSchedThreads) {
     int b, pr, cost;
     if (!block_of(g, b, pr, cost)) continue;
     const int pos = atomicAdd(&hist[cost < nbins ? cost : nbins - 1], a.H);

@@ -158,10 +158,10 @@ hstu_status_t hstu_attn_fwd_rab(const void* q, const void* k, const void* v,
  *   Layout (all int32, little endian):
  *     header[4]          {work counter, num_items, finished-CTA counter, 0}
  *     q_start[B]         first query row of each user (-1: user skipped), padded to 16 bytes
- *     pair_start[B+1]    index of each user's first 256-row block, padded to 16 bytes
- *     items[cap][4]      {b, pair, h, cost}, cap = H * (total_q / 256 + B); the first
- *                        num_items entries are valid, in non-increasing cost order.  `pair` is
- *                        a block of 256 query rows of user b; `cost` is the number of 128x128
+ *     block_start[B+1]   index of each user's first 128-row block, padded to 16 bytes
+ *     items[cap][4]      {b, block, h, cost}, cap = H * (total_q / 128 + B); the first
+ *                        num_items entries are valid, in non-increasing cost order.  `block` is
+ *                        a block of 128 query rows of user b; `cost` is the number of 128x128
  *                        score tiles the block computes (fully masked tiles are not counted).
  *
  * hstu_attn_plan — validates the offsets on the device and writes the plan.
@@ -205,7 +205,7 @@ hstu_status_t hstu_attn_fwd_planned(const void* q, const void* k, const void* v,
  *   Arguments are those of hstu_attn_fwd_cached (cached_len = NULL and total_q = total_kv for a
  *   full pass).  The caller still provides q, k, v and out.
  *   Limit: hstu_attn_plan_bytes(B, H, total_q) must not exceed HSTU_ATTN_NOALLOC_PLAN_BYTES
- *   (1 MiB: about 65,000 work items of 256 query rows x 1 head, e.g. H = 8 and 2 million query
+ *   (1 MiB: about 65,000 work items of 128 query rows x 1 head, e.g. H = 8 and 1 million query
  *   rows); larger batches return HSTU_ERR_UNSUPPORTED before anything is launched.
  *   Memory: every GPU that loads the library holds the 1 MiB array until the process exits.
  *   First call: the first call on each device (with that device current) looks up the array's

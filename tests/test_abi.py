@@ -46,7 +46,7 @@ def test_status_strings(cuda_lib):
 def test_plan_bytes(cuda_lib):
     """16-byte header, B query-row starts and B+1 block starts (each padded to 16 bytes), 16 bytes
     per possible item."""
-    assert cuda_lib.hstu_attn_plan_bytes(8, 4, 32768) == 16 + 32 + 48 + 16 * 4 * (32768 // 256 + 8)
+    assert cuda_lib.hstu_attn_plan_bytes(8, 4, 32768) == 16 + 32 + 48 + 16 * 4 * (32768 // 128 + 8)
     assert cuda_lib.hstu_attn_plan_bytes(3, 1, 10) == 16 + 16 + 16 + 16 * 3
     assert cuda_lib.hstu_attn_plan_bytes(-1, 4, 10) == 0
 

@@ -28,17 +28,14 @@ def expected_items(seq_offsets, num_targets, cached_len, H):
         c = int(cached_len[b]) if cached_len is not None else 0
         U = L - T
         nq = L - c
-        for pair in range(0, (nq + 255) // 256):
-            cost = 0
-            for half in range(2):
-                r0 = pair * 256 + half * 128
-                r1 = min(r0 + 128, nq)
-                tiles = set()
-                for r in range(r0, r1):
-                    tiles |= {j // 128 for j in visible_keys(c + r, U, L)}
-                cost += len(tiles)
+        for blk in range(0, (nq + 127) // 128):
+            r0 = blk * 128
+            r1 = min(r0 + 128, nq)
+            tiles = set()
+            for r in range(r0, r1):
+                tiles |= {j // 128 for j in visible_keys(c + r, U, L)}
             for h in range(H):
-                items.append((b, pair, h, cost))
+                items.append((b, blk, h, len(tiles)))
     return items
 
 
