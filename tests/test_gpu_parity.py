@@ -3,7 +3,7 @@ bf16 inputs.  Bar (bf16 inputs N(0,1)/sqrt(d)): relative L2 error <= 5e-3 and ma
 <= 3e-2 over the compared outputs.
 
 - small jagged batches are compared element by element over every output row: ragged lengths
-  around the 128-row tiles and 256-row work items, zero-length users, no-history users,
+  around the 128-row tiles and work items, zero-length users, no-history users,
   candidate-only users, single tokens, every head size;
 - the four large named workloads run at full size in the bench's launch configuration and are
   compared on sampled rows (tile edges, the history/candidate boundary, both ends, random rows);
