@@ -10,7 +10,7 @@ are re-exported lazily so that :mod:`.workloads` and :mod:`.metrics` import with
 """
 _BINDING_NAMES = ("HstuError", "hstu_attn_fwd", "hstu_attn_fwd_cached", "hstu_attn_fwd_rab", "hstu_attn_plan_bytes", "hstu_attn_plan",
                   "hstu_attn_fwd_planned", "hstu_attn_fwd_noalloc", "hstu_attn_get_error", "hstu_attn_status_string",
-                  "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16", "hstu_attn_bwd", "hstu_attn_partition", "shard_of", "hstu_layer_workspace_bytes",
+                  "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16", "hstu_attn_bwd", "hstu_attn_bwd_workspace_limit", "hstu_attn_partition", "shard_of", "hstu_layer_workspace_bytes",
                   "hstu_layer_fwd", "hstu_layers_fwd", "plan_contents",
                   "library_path", "load_library")
 

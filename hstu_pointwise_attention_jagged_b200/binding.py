@@ -37,6 +37,7 @@ EXPORTS = (
     "hstu_attn_selfcheck_wait_timeout",
     "hstu_attn_gemm_bf16",
     "hstu_attn_bwd",
+    "hstu_attn_bwd_workspace_limit",
     "hstu_attn_partition",
     "hstu_layer_workspace_bytes",
     "hstu_layer_fwd",
@@ -85,6 +86,8 @@ def load_library():
     lib.hstu_attn_selfcheck_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.hstu_attn_gemm_bf16.argtypes = [vp, vp, vp, i32, i32, i32, vp]
     lib.hstu_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp, vp]
+    lib.hstu_attn_bwd_workspace_limit.argtypes = [ctypes.c_uint64]
+    lib.hstu_attn_bwd_workspace_limit.restype = ctypes.c_uint64
     lib.hstu_attn_partition.argtypes = [vp, vp, vp, i32, i32, vp]
     lib.hstu_attn_selfcheck_fwd_timeout.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp,
                                                     ctypes.c_uint64, vp]
@@ -368,6 +371,12 @@ def hstu_attn_bwd(q, k, v, dout, seq_offsets, num_targets, alpha, N, max_seq_len
                                _stream_ptr(stream, q.device))
     _raise_if(st, "hstu_attn_bwd")
     return dq, dk, dv
+
+
+def hstu_attn_bwd_workspace_limit(max_bytes):
+    """Largest dS workspace (bytes) hstu_attn_bwd may take per call (0: recompute dS for dq); returns
+    the previous limit. See include/hstu_attn.h."""
+    return int(load_library().hstu_attn_bwd_workspace_limit(int(max_bytes)))
 
 
 def hstu_attn_partition(seq_offsets, num_targets, cached_len, parts):

@@ -33,12 +33,26 @@ __host__ __device__ __forceinline__ TileRange key_tiles_of_query_tile(int qt, in
   return key_tiles(p0, p1, U);
 }
 
+// dS tiles of one head of a segment, kept for the dQ pass: one 128 x 128 tile per visible (key
+// tile, query tile) pair, in key-tile order.  A history key tile kt pairs with query tiles
+// kt .. T-1, a candidate-only key tile with its own query tile, so tile (kt, qt) sits at
+// ds_tiles_before(kt) + (qt - kt).
+__host__ __device__ __forceinline__ long long ds_tiles_before(int kt, int L, int U) {
+  const long long T = cdiv(L, kTileRows), Th = cdiv(U, kTileRows), k = kt;
+  if (k <= Th) return k * T - k * (k - 1) / 2;
+  return Th * T - Th * (Th - 1) / 2 + (k - Th);
+}
+__host__ __device__ __forceinline__ long long ds_tiles_per_head(int L, int U) {
+  return ds_tiles_before(cdiv(L, kTileRows), L, U);
+}
+
 struct BwdSchedArgs {
   const int32_t* seq_offsets;  // [B+1]
   const int32_t* num_targets;  // [B] or null
   int32_t B, H, total, max_seq_len, nbins, max_items;
   int32_t* header;      // [8] out: {dq counter, dq items, dq done, 0, kv counter, kv items, kv done, 0}
   int32_t* tile_start;  // [B+1] out: index of each user's first 128-row tile among all tiles
+  long long* ds_base;   // [B+1] out: index of each user's first dS tile (all heads); may be null
   int4* dq_items;       // [max_items] out: {b, query tile, h, cost}, non-increasing cost
   int4* kv_items;       // [max_items] out: {b, key tile, h, cost}, non-increasing cost
   unsigned* err;
@@ -50,18 +64,18 @@ __global__ void __launch_bounds__(kSchedThreads) bwd_schedule_kernel(const BwdSc
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ int hist[kMaxCostBins];
   __shared__ long long scan_scratch[2][32];
-  __shared__ long long carry;
+  __shared__ long long carry, carry_ds;
   __shared__ int s_L[kCachedUsers], s_U[kCachedUsers], s_ts[kCachedUsers + 1];
   const bool cached = a.B <= kCachedUsers;
   const int tid = threadIdx.x;
   const int nbins = a.nbins;
-  if (tid == 0) carry = 0;
+  if (tid == 0) carry = carry_ds = 0;
   __syncthreads();
 
   // Pass 1: validation and tile starts.
   for (int base = 0; base < a.B; base += kSchedThreads) {
     const int b = base + tid;
-    long long nt = 0, dummy = 0;
+    long long nt = 0, nds = 0;
     int L = 0, U = 0;
     if (b < a.B) {
       const int o0 = a.seq_offsets[b], o1 = a.seq_offsets[b + 1];
@@ -74,12 +88,14 @@ __global__ void __launch_bounds__(kSchedThreads) bwd_schedule_kernel(const BwdSc
       L = ok ? (int)L64 : 0;
       U = L - (ok ? T : 0);
       nt = cdiv(L, kTileRows);
+      nds = ds_tiles_per_head(L, U);
     }
-    long long incl = nt, tot, tot2;
-    block_inclusive_scan2(incl, dummy, scan_scratch, tot, tot2);
+    long long incl = nt, incl_ds = nds, tot, tot_ds;
+    block_inclusive_scan2(incl, incl_ds, scan_scratch, tot, tot_ds);
     const long long start = carry + incl - nt;
     if (b < a.B) {
       a.tile_start[b] = (int)start;
+      if (a.ds_base) a.ds_base[b] = (carry_ds + incl_ds - nds) * a.H;
       if (cached) {
         s_L[b] = L;
         s_U[b] = U;
@@ -87,12 +103,16 @@ __global__ void __launch_bounds__(kSchedThreads) bwd_schedule_kernel(const BwdSc
       }
     }
     __syncthreads();
-    if (tid == 0) carry += tot;
+    if (tid == 0) {
+      carry += tot;
+      carry_ds += tot_ds;
+    }
     __syncthreads();
   }
   const int ntiles = (int)carry;
   if (tid == 0) {
     a.tile_start[a.B] = ntiles;
+    if (a.ds_base) a.ds_base[a.B] = carry_ds * a.H;
     if (cached) s_ts[a.B] = ntiles;
   }
   __syncthreads();

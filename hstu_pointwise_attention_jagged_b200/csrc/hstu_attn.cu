@@ -12,11 +12,13 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <functional>
 #include <mutex>
 #include <vector>
 
 #include "hstu_attn.h"
+#include "hstu_bwd_dq_sm100.cuh"
 #include "hstu_bwd_sm100.cuh"
 #include "hstu_fwd_sm100.cuh"
 #include "gemm_sm100.cuh"
@@ -56,6 +58,9 @@ cudaError_t set_kernel_attrs() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(hstu_bwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              BwdCfg<D>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(hstu_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DqCfg<D>::kSmemBytes);
   return e;
 }
 
@@ -410,14 +415,31 @@ hstu_status_t run(const void* q, const void* k, const void* v, const int32_t* se
 // Backward plan layout:
 //   int32 header[8] = {dq counter, dq items, dq done, 0, kv counter, kv items, kv done, 0}
 //   int32 tile_start[B+1], padded to 16 bytes
+//   int64 ds_base[B+1], padded to 16 bytes
 //   int4  dq_items[cap], kv_items[cap], cap = H * (total / 128 + B)
 int64_t bwd_capacity(int32_t B, int32_t H, int32_t total) {
   return static_cast<int64_t>(H) * (total / kTileRows + B);
 }
 
+size_t pad16_64(size_t n) { return ((n * 8 + 15) / 16) * 16; }
+
 int64_t bwd_plan_bytes(int32_t B, int32_t H, int32_t total) {
-  return 32 + static_cast<int64_t>(pad16(static_cast<size_t>(B) + 1)) + 2 * bwd_capacity(B, H, total) * 16;
+  return 32 + static_cast<int64_t>(pad16(static_cast<size_t>(B) + 1) + pad16_64(static_cast<size_t>(B) + 1)) +
+         2 * bwd_capacity(B, H, total) * 16;
 }
+
+// dS workspace of the dQ pass, in 128 x 128 tiles: an upper bound on sum over users of
+// H * ds_tiles_per_head, from sizes the host knows.  A user of T tiles holds at most
+// T (T + 1) / 2 pairs per head, T <= max_seq_len / 128 + 1 and the users' T sum to at most
+// total / 128 + B.
+int64_t bwd_ds_tiles_bound(int32_t B, int32_t H, int32_t total, int32_t max_seq_len) {
+  const int64_t sum_t = static_cast<int64_t>(total) / kTileRows + B;
+  const int64_t max_t = static_cast<int64_t>(max_seq_len) / kTileRows + 1;
+  return static_cast<int64_t>(H) * (sum_t * (max_t + 1) / 2 + sum_t);
+}
+
+constexpr int64_t kDsTileBytes = static_cast<int64_t>(kTileRows) * kTileRows * 2;
+std::atomic<uint64_t> g_bwd_ds_limit{16ull << 30};  // bytes; 0: always recompute dS in the dQ pass
 
 // Both backward kernels over a plan written by bwd_schedule_kernel.  Arguments already checked.
 template <int D, bool kDQ>
@@ -438,12 +460,32 @@ cudaError_t launch_bwd_kernel(const CUtensorMap& f0, const CUtensorMap& f1, cons
 }
 
 template <int D>
+cudaError_t launch_bwd_dq(const CUtensorMap& tds, const CUtensorMap& tk, const DqParams& p, int grid,
+                          cudaStream_t stream) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kDqThreads);
+  cfg.dynamicSmemBytes = DqCfg<D>::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, hstu_bwd_dq_kernel<D>, tds, tk, p);
+}
+
+// dK/dV, then dQ: from the stored dS tiles when a workspace is given (tds valid), otherwise by
+// recomputing S, dP and dS.
+template <int D>
 cudaError_t launch_bwd_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, BwdParams pkv, BwdParams pq, int grid_kv, int grid_q,
-                            cudaStream_t stream) {
+                            const CUtensorMap& tdo, const CUtensorMap* tds, BwdParams pkv, BwdParams pq,
+                            const DqParams& pdq, int grid_kv, int grid_q, cudaStream_t stream) {
   cudaError_t e = launch_bwd_kernel<D, false>(tk, tv, tq, tdo, pkv, grid_kv, stream);
-  if (e == cudaSuccess) e = launch_bwd_kernel<D, true>(tq, tdo, tk, tv, pq, grid_q, stream);
-  return e;
+  if (e != cudaSuccess) return e;
+  return tds ? launch_bwd_dq<D>(*tds, tk, pdq, grid_q, stream)
+             : launch_bwd_kernel<D, true>(tq, tdo, tk, tv, pq, grid_q, stream);
 }
 
 hstu_status_t run_bwd(const void* q, const void* k, const void* v, const void* dout, const int32_t* seq_offsets,
@@ -484,9 +526,27 @@ hstu_status_t run_bwd(const void* q, const void* k, const void* v, const void* d
   uint8_t* pb = static_cast<uint8_t*>(plan);
   int32_t* header = reinterpret_cast<int32_t*>(pb);
   int32_t* tile_start = reinterpret_cast<int32_t*>(pb + 32);
+  long long* ds_base = reinterpret_cast<long long*>(pb + 32 + pad16(static_cast<size_t>(B) + 1));
   const int64_t cap = bwd_capacity(B, H, total);
-  int4* dq_items = reinterpret_cast<int4*>(pb + 32 + pad16(static_cast<size_t>(B) + 1));
+  int4* dq_items = reinterpret_cast<int4*>(pb + 32 + pad16(static_cast<size_t>(B) + 1) +
+                                           pad16_64(static_cast<size_t>(B) + 1));
   int4* kv_items = dq_items + cap;
+  // The dS workspace, when its bound fits the limit and the pool has the memory; otherwise the dQ
+  // pass recomputes dS.
+  const int64_t ds_tiles = bwd_ds_tiles_bound(B, H, total, max_seq_len);
+  void* ds_ws = nullptr;
+  CUtensorMap tds;
+  if (ds_tiles > 0 && ds_tiles * kTileRows <= INT_MAX &&
+      static_cast<uint64_t>(ds_tiles * kDsTileBytes) <= g_bwd_ds_limit.load()) {
+    if (cudaMallocFromPoolAsync(&ds_ws, static_cast<size_t>(ds_tiles * kDsTileBytes), st->pool, stream) !=
+        cudaSuccess) {
+      ds_ws = nullptr;
+      cudaGetLastError();  // an allocation the pool cannot serve is not an error of the call
+    } else if (!encode_matrix(&tds, ds_ws, ds_tiles * kTileRows, kTileRows, kTileRows)) {
+      cudaFreeAsync(ds_ws, stream);
+      ds_ws = nullptr;
+    }
+  }
   BwdSchedArgs a;
   a.seq_offsets = seq_offsets;
   a.num_targets = num_targets;
@@ -498,6 +558,7 @@ hstu_status_t run_bwd(const void* q, const void* k, const void* v, const void* d
   a.max_items = static_cast<int32_t>(cap);
   a.header = header;
   a.tile_start = tile_start;
+  a.ds_base = ds_base;
   a.dq_items = dq_items;
   a.kv_items = kv_items;
   a.err = st->err_word;
@@ -518,20 +579,37 @@ hstu_status_t run_bwd(const void* q, const void* k, const void* v, const void* d
     pkv.ds_scale = 0.5f * alpha / N;
     pkv.inv_n = 1.0f / N;
     pkv.err = st->err_word;
+    pkv.ds_ws = static_cast<__nv_bfloat16*>(ds_ws);
+    pkv.ds_base = ds_base;
+    pkv.ds_cap = ds_ws ? ds_tiles : 0;
     BwdParams pq = pkv;
+    pq.ds_ws = nullptr;
     pq.items = dq_items;
     pq.num_items = header + 1;
     pq.work_counter = header + 0;
     pq.done_counter = header + 2;
     pq.out0 = static_cast<__nv_bfloat16*>(dq);
     pq.out1 = nullptr;
+    DqParams pdq;
+    pdq.seq_offsets = seq_offsets;
+    pdq.num_targets = num_targets;
+    pdq.items = dq_items;
+    pdq.num_items = header + 1;
+    pdq.work_counter = header + 0;
+    pdq.done_counter = header + 2;
+    pdq.ds_base = ds_base;
+    pdq.dq = static_cast<__nv_bfloat16*>(dq);
+    pdq.H = H;
+    pdq.err = st->err_word;
+    const CUtensorMap* tdsp = ds_ws ? &tds : nullptr;
     const int grid = static_cast<int>(cap < st->num_sms ? cap : st->num_sms);
     cudaError_t e;
-    if (d == 128) e = launch_bwd_pair<128>(tq, tk, tv, tdo, pkv, pq, grid, grid, stream);
-    else if (d == 64) e = launch_bwd_pair<64>(tq, tk, tv, tdo, pkv, pq, grid, grid, stream);
-    else e = launch_bwd_pair<32>(tq, tk, tv, tdo, pkv, pq, grid, grid, stream);
+    if (d == 128) e = launch_bwd_pair<128>(tq, tk, tv, tdo, tdsp, pkv, pq, pdq, grid, grid, stream);
+    else if (d == 64) e = launch_bwd_pair<64>(tq, tk, tv, tdo, tdsp, pkv, pq, pdq, grid, grid, stream);
+    else e = launch_bwd_pair<32>(tq, tk, tv, tdo, tdsp, pkv, pq, pdq, grid, grid, stream);
     if (e != cudaSuccess) s = HSTU_ERR_CUDA;
   }
+  if (ds_ws && cudaFreeAsync(ds_ws, stream) != cudaSuccess && s == HSTU_OK) s = HSTU_ERR_CUDA;
   if (cudaFreeAsync(plan, stream) != cudaSuccess && s == HSTU_OK) s = HSTU_ERR_CUDA;
   return s;
 }
@@ -605,6 +683,8 @@ hstu_status_t hstu_attn_fwd_rab(const void* q, const void* k, const void* v, con
   return hstu::run(q, k, v, seq_offsets, num_targets, cached_len, B, H, d, total_kv, total_q, max_seq_len, alpha,
                    N, out, stream, rab, rab_len);
 }
+
+uint64_t hstu_attn_bwd_workspace_limit(uint64_t max_bytes) { return hstu::g_bwd_ds_limit.exchange(max_bytes); }
 
 hstu_status_t hstu_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
                             const int32_t* seq_offsets, const int32_t* num_targets, int32_t B, int32_t H, int32_t d,

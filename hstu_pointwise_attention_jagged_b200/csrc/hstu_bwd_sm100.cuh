@@ -66,6 +66,11 @@ struct BwdParams {
   float ds_scale;       // alpha / (2 N)
   float inv_n;
   unsigned* err;
+  // dK/dV kernel, when the dQ pass reads dS instead of recomputing it: the dS workspace (ds_cap
+  // tiles of 128 x 128 bf16, row-major [key][query]) and each user's first tile (plan).
+  __nv_bfloat16* ds_ws;
+  const long long* ds_base;
+  long long ds_cap;
 };
 
 template <int kStages>
@@ -86,6 +91,7 @@ struct BwdCtl {
 struct BwdWork {
   int valid, h, row0, fixed, L, U;
   TileRange r;
+  int b;
 };
 
 __device__ __forceinline__ BwdWork read_bwd_slot(const volatile int32_t* s) {
@@ -99,6 +105,7 @@ __device__ __forceinline__ BwdWork read_bwd_slot(const volatile int32_t* s) {
   w.r.e1 = s[6];
   w.r.s2 = s[7];
   w.r.e2 = s[8];
+  w.b = s[9];
   return w;
 }
 
@@ -140,7 +147,7 @@ __device__ __forceinline__ void bwd_scores(const uint32_t (&s)[32], float (&m)[3
 // Second half: dS = (dP ds_scale) m, an exact zero outside the visible columns, packed as bf16
 // pairs into 16 TMEM columns.
 __device__ __forceinline__ void bwd_grads(const uint32_t (&dp)[32], const float (&m)[32], uint32_t t_ds,
-                                          float ds_scale, bool full, int lo, int hi, int self) {
+                                          float ds_scale, bool full, int lo, int hi, int self, uint4* g_ds) {
   uint32_t pk[16];
   const uint64_t sc2 = ptx::f32x2(ds_scale, ds_scale);
 #pragma unroll
@@ -157,6 +164,11 @@ __device__ __forceinline__ void bwd_grads(const uint32_t (&dp)[32], const float 
     pk[e] = pack_bf16x2(d0, d1);
   }
   ptx::tmem_st16(t_ds, pk);
+  if (g_ds != nullptr) {
+    // The same 32 values into the dS workspace for the dQ pass (written once, read by another kernel).
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) g_ds[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+  }
 }
 
 template <int D, bool kDQ>
@@ -231,6 +243,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (w.valid) {
           const int4 it = p.items[idx];
           const int b = it.x;
+          w.b = b;
           w.fixed = it.y;
           w.h = it.z;
           w.row0 = p.seq_offsets[b];
@@ -242,7 +255,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         sched_empty_par[slot] ^= 1u;
         volatile int32_t* s = ctl->slot[slot];
         s[0] = w.valid; s[1] = w.h; s[2] = w.row0; s[3] = w.fixed; s[4] = w.L; s[5] = w.U;
-        s[6] = w.r.e1; s[7] = w.r.s2; s[8] = w.r.e2;
+        s[6] = w.r.e1; s[7] = w.r.s2; s[8] = w.r.e2; s[9] = w.b;
         ptx::mbar_arrive(bar(ctl->sched_full[slot]));
         slot ^= 1;
         if (!w.valid) break;
@@ -466,7 +479,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(ctl->p_full));
-        // Second half: dP -> dS over dP.
+        // Second half: dP -> dS over dP (and, for the dQ pass, into the workspace: tile (key tile
+        // w.fixed, query tile w.fixed + i) of this user and head, this thread's row and 64 columns).
+        uint4* g_ds = nullptr;
+        if constexpr (!kDQ) {
+          if (p.ds_ws != nullptr) {
+            const long long tile = p.ds_base[w.b] + (long long)w.h * ds_tiles_per_head(w.L, w.U) +
+                                   ds_tiles_before(w.fixed, w.L, w.U) + i;
+            if (tile < p.ds_cap)
+              g_ds = reinterpret_cast<uint4*>(p.ds_ws + (tile * kTileRows + row) * kTileRows + 64 * ch);
+            else if (lane == 0)
+              atomicOr(p.err, kErrBadOffsets);  // the workspace bound was wrong: report, write nothing
+          }
+        }
         ok = __all_sync(0xffffffffu, wait_bounded(bar(ctl->dp_full), dp_full_par, abort_flag, p.err));
         if (!ok) break;
         dp_full_par ^= 1u;
@@ -476,7 +501,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t rd[32];
           ptx::tmem_ld32(t_dp + 32 * k, rd);
           ptx::tmem_ld_wait(rd);
-          bwd_grads(rd, m[k], t_dp + 16 * k, p.ds_scale, full, lo - 32 * k, hi - 32 * k, self - 32 * k);
+          bwd_grads(rd, m[k], t_dp + 16 * k, p.ds_scale, full, lo - 32 * k, hi - 32 * k, self - 32 * k,
+                    g_ds ? g_ds + 4 * k : nullptr);
         }
         ptx::tmem_st_wait();
         ptx::tc_fence_before();

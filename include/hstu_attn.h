@@ -251,6 +251,11 @@ hstu_status_t hstu_attn_fwd_noalloc(const void* q, const void* k, const void* v,
  *   stream          cudaStream_t as void*.
  * A stream-ordered plan buffer is taken from the library's pool and returned, as in
  * hstu_attn_fwd.  Errors as in hstu_attn_fwd; inputs must be finite (as there).
+ * Workspace: the dK/dV kernel forms every bf16 dS tile; when a workspace for them fits the limit
+ * set by hstu_attn_bwd_workspace_limit (2 bytes per visible pair and head, sized on the host from
+ * an upper bound in total_tokens, B, H and max_seq_len), it keeps them there, stream-ordered from
+ * the pool, and dq is a plain product of them with k.  Otherwise the dQ kernel recomputes them.
+ * Both ways give the same gradients.
  */
 hstu_status_t hstu_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
                             const int32_t* seq_offsets, const int32_t* num_targets,
@@ -258,6 +263,13 @@ hstu_status_t hstu_attn_bwd(const void* q, const void* k, const void* v, const v
                             int32_t total_tokens, int32_t max_seq_len,
                             float alpha, float N,
                             void* dq, void* dk, void* dv, void* stream);
+
+/*
+ * hstu_attn_bwd_workspace_limit — sets the largest dS workspace (bytes) hstu_attn_bwd may take
+ * from the pool for one call, and returns the previous limit.  Default 16 GiB; 0 makes every call
+ * recompute dS in its dQ kernel.  Process-wide; takes effect for calls made after it returns.
+ */
+uint64_t hstu_attn_bwd_workspace_limit(uint64_t max_bytes);
 
 /*
  * hstu_attn_partition — splits one jagged batch across `parts` GPUs (host function, no GPU work).

@@ -22,7 +22,8 @@ def test_header_declares_the_entry_points():
                                            "hstu_attn_plan", "hstu_attn_fwd_planned", "hstu_attn_fwd_noalloc",
                                            "hstu_attn_get_error", "hstu_attn_status_string",
                                            "hstu_attn_selfcheck_wait_timeout", "hstu_attn_gemm_bf16",
-                                           "hstu_attn_bwd", "hstu_attn_partition", "hstu_layer_workspace_bytes",
+                                           "hstu_attn_bwd", "hstu_attn_bwd_workspace_limit", "hstu_attn_partition",
+                                           "hstu_layer_workspace_bytes",
                                            "hstu_layer_fwd", "hstu_layers_fwd", "hstu_attn_selfcheck_fwd_timeout"])
 
 

@@ -103,3 +103,28 @@ def test_bwd_deterministic_and_guarded():
         assert torch.equal(x, y)
         assert torch.all(big[:pad] == 7.0) and torch.all(big[pad + w.total:] == 7.0)
     assert binding.hstu_attn_get_error() == 0
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_bwd_stored_ds_path_matches_recompute_path(d):
+    """hstu_attn_bwd with its dS workspace (dq from the stored dS tiles) and with the workspace limit
+    at 0 (the dQ kernel recomputes S, dP and dS): both match the oracle, dk and dv are bitwise
+    equal (same kernel), and the two dq agree to fp32 accumulation order."""
+    uih, nt = RAGGED[1]
+    w = workloads.make_custom("bwdws%d" % d, uih, nt, 2, d, 1 / math.sqrt(d),
+                              float(max(u + t for u, t in zip(uih, nt))), seed=500 + d)
+    do = _dout(w, 600 + d)
+    stored = _run(w, do)
+    previous = binding.hstu_attn_bwd_workspace_limit(0)
+    try:
+        recomputed = _run(w, do)
+    finally:
+        binding.hstu_attn_bwd_workspace_limit(previous)
+    assert binding.hstu_attn_get_error() == 0
+    want = oracle.bwd(w.q, w.k, w.v, do, w.seq_offsets, w.num_targets, w.alpha, w.N)
+    for path, got in (("stored dS", stored), ("recomputed dS", recomputed)):
+        for name, g, r in zip(("dq", "dk", "dv"), got, want):
+            assert_parity(to_f64(g), r, what="bwd %s %s d=%d" % (name, path, d), users=row_users(w))
+    assert torch.equal(stored[1], recomputed[1]) and torch.equal(stored[2], recomputed[2])
+    a, b = stored[0].double(), recomputed[0].double()
+    assert float((a - b).norm() / b.norm()) <= 1e-2 * 2.0 ** -8  # a few bf16 ulps at most, by accumulation order
