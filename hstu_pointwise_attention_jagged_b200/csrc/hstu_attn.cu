@@ -37,6 +37,7 @@ struct DeviceState {
   std::once_flag once;
   cudaError_t init_err = cudaSuccess;
   int num_sms = 0;
+  int gemm_clusters = 0;  // resident two-CTA clusters of the two-SM GEMM
   cudaMemPool_t pool = nullptr;
   unsigned* err_word = nullptr;
 };
@@ -87,6 +88,25 @@ void init_device(DeviceState& st, int dev) {
   if (e == cudaSuccess) e = set_kernel_attrs<128>();
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_bf16_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Gemm2Cfg::kSmemBytes);
+  if (e == cudaSuccess) {
+    // How many two-CTA clusters of the two-SM GEMM can be resident at once (SM pairs with room).
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (st.num_sms / 2));
+    cfg.blockDim = dim3(kGemm2Threads);
+    cfg.dynamicSmemBytes = Gemm2Cfg::kSmemBytes;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaOccupancyMaxActiveClusters(&st.gemm_clusters, gemm_bf16_2sm_kernel, &cfg);
+  }
   st.init_err = e;
 }
 
@@ -316,8 +336,8 @@ hstu_status_t launch_attention(DeviceState* st, const void* q, const void* k, co
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
-// C = A W^T on the projection GEMM kernel.  Arguments already checked.
-hstu_status_t launch_gemm(DeviceState* st, const void* a, const void* w, void* c, int32_t M, int32_t N, int32_t K,
+// C = A W^T on the one-SM projection GEMM kernel (128 × 256 tiles).  Arguments already checked.
+hstu_status_t launch_gemm_1sm(DeviceState* st, const void* a, const void* w, void* c, int32_t M, int32_t N, int32_t K,
                           cudaStream_t stream) {
   if (!encoder()) return HSTU_ERR_CUDA;
   CUtensorMap ta, tw;
@@ -335,6 +355,47 @@ hstu_status_t launch_gemm(DeviceState* st, const void* a, const void* w, void* c
   const int grid = static_cast<int>(ntiles < st->num_sms ? ntiles : st->num_sms);
   gemm_bf16_kernel<<<grid, kGemmThreads, GemmCfg::kSmemBytes, stream>>>(ta, tw, p);
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// The same product on the two-SM kernel: 256 × 256 tiles, one per cluster of two CTAs.
+hstu_status_t launch_gemm_2sm(DeviceState* st, const void* a, const void* w, void* c, int32_t M, int32_t N,
+                              int32_t K, cudaStream_t stream) {
+  if (!encoder()) return HSTU_ERR_CUDA;
+  CUtensorMap ta, tw;
+  if (!encode_matrix(&ta, a, M, K, 128) || !encode_matrix(&tw, w, N, K, 128)) return HSTU_ERR_CUDA;
+  GemmParams p;
+  p.c = static_cast<__nv_bfloat16*>(c);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.tiles_m = (M + kGemm2BM - 1) / kGemm2BM;
+  p.tiles_n = (N + kGemm2BN - 1) / kGemm2BN;
+  p.err = st->err_word;
+  const int64_t ntiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+  if (ntiles > INT_MAX / 2) return HSTU_ERR_UNSUPPORTED;
+  const int clusters = static_cast<int>(ntiles < st->gemm_clusters ? ntiles : st->gemm_clusters);
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(kGemm2Threads);
+  cfg.dynamicSmemBytes = Gemm2Cfg::kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_bf16_2sm_kernel, ta, tw, p) == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// C = A W^T: the two-SM kernel once A has a full 256-row tile, the one-SM kernel below that (or
+// when no SM pair can hold a cluster).  Arguments already checked.
+hstu_status_t launch_gemm(DeviceState* st, const void* a, const void* w, void* c, int32_t M, int32_t N, int32_t K,
+                          cudaStream_t stream) {
+  if (M >= kGemm2BM && st->gemm_clusters > 0) return launch_gemm_2sm(st, a, w, c, M, N, K, stream);
+  return launch_gemm_1sm(st, a, w, c, M, N, K, stream);
 }
 
 // One HSTU layer over a plan built for its offsets (full sequences):

@@ -45,9 +45,11 @@ def test_gemm_layer_projection_shapes(shape):
     assert torch.isfinite(c.float()).all()
 
 
-def test_gemm_writes_nothing_outside_c():
-    """Guard rows around C stay untouched (row- and column-predicated stores)."""
-    M, N, K = 200, 264, 128
+@pytest.mark.parametrize("M", [200, 300])
+def test_gemm_writes_nothing_outside_c(M):
+    """Guard rows around C stay untouched (row- and column-predicated stores); M = 200 runs the one-SM
+    kernel, M = 300 the two-SM kernel with a ragged last tile."""
+    N, K = 264, 128
     a, w = _mats(M, N, K, seed=9)
     buf = torch.full((M + 2, N), 7.0, dtype=torch.bfloat16, device="cuda")
     binding.hstu_attn_gemm_bf16(_dev(a), _dev(w), out=buf[1:M + 1])
