@@ -254,9 +254,6 @@ constexpr int kGemm2BN = 256;  // rows of W per cluster tile (128 per CTA)
 constexpr int kGemm2Stages = 6;
 constexpr int kGemm2EpiWarps = 4;
 constexpr int kGemm2Threads = 64 + 32 * kGemm2EpiWarps;
-// On the abort path CTA 1 cannot wait on the barrier its copies complete on (it lives in CTA 0),
-// so it gives them this long to land (a copy takes microseconds) before it leaves.
-constexpr uint64_t kPeerCopyGraceNs = 1000000ull;
 
 struct Gemm2Cfg {
   static constexpr int kHalfBytes = 128 * kGemmBK * 2;  // 16 KB: 128 rows × 64 of A or of W
@@ -371,8 +368,10 @@ __global__ void __launch_bounds__(kGemm2Threads, 1)
             drain_wait(bar(ctl->full[pos % kGemm2Stages]), (uint32_t)((pos / kGemm2Stages) & 1));
           }
         } else {
+          // CTA 1 cannot wait on the barrier its copies complete on (it lives in CTA 0), so it
+          // gives them kCopyGraceNs to land (a copy takes microseconds) before it leaves.
           const uint64_t t0 = ptx::globaltimer_ns();
-          while (ptx::globaltimer_ns() - t0 < kPeerCopyGraceNs) {
+          while (ptx::globaltimer_ns() - t0 < kCopyGraceNs) {
           }
         }
       }

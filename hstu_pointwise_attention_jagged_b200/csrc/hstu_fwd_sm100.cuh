@@ -87,6 +87,7 @@ constexpr int kEpiWarp0 = 10;     // first of the four epilogue warps
 constexpr int kSlots = 4;         // work-item slots between the producer and the other roles
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s per wait
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s per drain wait on the abort path
+constexpr uint64_t kCopyGraceNs = 1000000ull;     // 1 ms for the copies in flight on the abort path
 
 struct FwdParams {
   const int32_t* seq_offsets;
@@ -412,14 +413,21 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         armed_hi = t + 4;
       }
       if (*abort_flag) {
-        // Let every copy this CTA started land before its shared memory is released: each group
-        // barrier still in use gets the SiLU arrivals that may never come (extra ones only spill
-        // into a phase nobody waits for), then its bytes are awaited.
+        // Let every copy this CTA started land before its shared memory is released.  A group
+        // barrier's phase completes once its bytes and the SiLU warps' arrivals are in, and the
+        // arrivals of an aborted group may never come.  Arriving for them here is not an option:
+        // if they did come while bytes were still outstanding, the extra arrival would land on a
+        // phase with no arrivals pending, which is not defined.  So the producer only waits, on
+        // each barrier still in use, all within one budget of kCopyGraceNs: every phase complete
+        // means every copy landed, and otherwise the whole budget, a thousand times a copy's
+        // duration, has passed.
+        const uint64_t t0 = ptx::globaltimer_ns();
         for (int x = armed_hi > kGroupBars ? armed_hi - kGroupBars : 0; x < armed_hi; ++x) {
           if (x >= g && x < 3) continue;  // group indices never used when the CTA had < 3 tiles
           const uint32_t rb = bar(ctl->g_ready[x & (kGroupBars - 1)]);
-          for (int a = 0; a < 4; ++a) ptx::mbar_arrive(rb);
-          drain_wait(rb, (uint32_t)((x / kGroupBars) & 1));
+          const uint32_t par = (uint32_t)((x / kGroupBars) & 1);
+          while (!ptx::mbar_test_wait(rb, par) && ptx::globaltimer_ns() - t0 < kCopyGraceNs) {
+          }
         }
       }
     }

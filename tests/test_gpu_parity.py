@@ -55,6 +55,25 @@ def test_ragged_batches(d, case):
     _full_compare(w, "ragged case %d d=%d" % (case, d))
 
 
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_candidate_own_pairs(d):
+    """Candidates at or past the first key tile that starts at or after U: the kernel does not
+    enumerate their own key tiles and adds each one's own pair in the epilogue.  History lengths on
+    and off the 128-row grid, several candidate tiles per user, the mixed tile that holds U, and a
+    cached form whose query tiles sit off the key-tile grid; every row against the oracle."""
+    uih, nt = [1, 128, 200, 383, 512, 0], [300, 129, 250, 400, 3, 140]
+    H = 3 if d == 32 else 2
+    N = float(max(u + t for u, t in zip(uih, nt)))
+    w = workloads.make_custom("own%d" % d, uih, nt, H, d, 1 / math.sqrt(d), N, seed=300 + d)
+    _full_compare(w, "candidate own pairs d=%d" % d)
+    wc = workloads.make_custom("ownc%d" % d, uih, nt, H, d, 1 / math.sqrt(d), N, seed=310 + d,
+                               cached_len=[0, 100, 150, 383, 500, 0])
+    got = to_f64(run_cached(wc))
+    ref = oracle.fwd_cached(wc.q[wc.new_rows()], wc.k, wc.v, wc.seq_offsets, wc.num_targets, wc.cached_len,
+                            wc.alpha, wc.N)
+    assert_parity(got, ref, what="candidate own pairs cached d=%d" % d, users=row_users(wc, cached=True))
+
+
 def test_plain_causal_without_num_targets():
     w = workloads.make_custom("causal", [200, 1, 77, 400], [0, 0, 0, 0], 2, 128, 1 / math.sqrt(128), 400.0, seed=7)
     got = to_f64(run_fwd(w, num_targets=None))

@@ -13,6 +13,9 @@ show that (1) group_of_load names the group that really consumed each load, (2) 
 reused before its previous tile was consumed, (3) no parity wait can see a barrier two phases
 ahead, for the ring depths the kernel uses (5 slots at d = 128, 10 at d <= 64), and (4) the
 constraint kStages <= 2 kSCommits - 2 stated beside the kernel's configuration is the exact limit.
+An event-level model of the group barriers then replays random interleavings of the roles, with
+and without an abort, to show that no arrival ever lands on a phase with no pending arrivals, and
+that the abort path's earlier stand-in arrivals could.
 """
 import numpy as np
 import pytest
@@ -102,3 +105,144 @@ def test_three_commit_barriers_would_not_cover_the_deep_ring():
         assert replay(200, 4)
     finally:
         K_SCOMMITS = saved
+
+
+# ---------------------------------------------------------------------------------------------
+# Event-level model of the group barriers, with an abort at a random moment.
+#
+# Group g of the MMA warp waits on g_ready[g mod 8]: the producer's expect-tx arrival plus the
+# bytes of the group's copies (Q on a query tile's first tile, V_{g-3}, K_g), and, for g >= 3, the
+# arrivals of the four SiLU warps that wrote P_{g-3} (the producer stands in for them when g < 3).
+# On abort every role leaves its loop; SiLU warps that already read a tile may still arrive, and
+# copies in flight still land.  The producer then lets its copies land before the CTA ends.
+#
+# An mbarrier arrival on a phase with no arrivals pending while bytes are still outstanding is not
+# defined; the model flags it.  An earlier drain added the four SiLU arrivals to each barrier still
+# in use and then waited for its phase, which can do exactly that when the SiLU warps did arrive.
+# The kernel's drain only waits (within a time budget, as a phase whose SiLU arrivals never come
+# cannot complete).
+# ---------------------------------------------------------------------------------------------
+class Barrier:
+    def __init__(self, count):
+        self.count, self.phase, self.pending, self.tx = count, 0, count, 0
+
+    def _maybe_complete(self):
+        if self.pending == 0 and self.tx == 0:
+            self.phase += 1
+            self.pending = self.count
+
+    def arrive(self, phase_expected, n=1, tx=0, check_phase=True):
+        for i in range(n):
+            if self.pending == 0:
+                raise AssertionError("arrival on a phase with no pending arrivals (bytes outstanding: %d)" % self.tx)
+            if check_phase:
+                assert self.phase == phase_expected, ("arrival for the wrong phase", self.phase, phase_expected)
+            self.pending -= 1
+            if i == 0:
+                self.tx += tx
+            self._maybe_complete()
+
+    def bytes_landed(self, nbytes):
+        self.tx -= nbytes
+        self._maybe_complete()
+
+    def done(self, phase):
+        return self.phase > phase
+
+
+def simulate(tiles, rng, abort_at=None, stand_in_on_abort=False, lag=2):
+    """One CTA's groups 0 .. tiles+2 under a random interleaving; returns the number of steps.
+    After an abort the producer's drain runs interleaved with the copies still landing and the
+    SiLU arrivals still to come."""
+    nbar = K_GROUP_BARS
+    bars = [Barrier(1 + 4) for _ in range(nbar)]
+    closing = list(range(max(tiles - 3, 0), tiles))
+    arm_order = list(range(tiles)) + [t + 3 for t in closing]  # groups in the order the producer arms them
+    armed, mma_next, in_flight, silu_todo = 0, 0, [], []
+    mma_done = set()
+    aborted, step = False, 0
+    drain, drain_i, drain_arrived = [], 0, False
+    while True:
+        step += 1
+        if abort_at is not None and step == abort_at:
+            aborted = True
+            drain = arm_order[max(armed - nbar, 0):armed]
+        actions = []
+        if not aborted and armed < len(arm_order):
+            # ring slots free once the group armed `lag` places earlier has completed
+            if armed - lag < 0 or arm_order[armed - lag] in mma_done:
+                actions.append("arm")
+        if not aborted and mma_next < len(arm_order):
+            x = arm_order[mma_next]
+            if bars[x % nbar].done(x // nbar):
+                actions.append("mma")
+        if in_flight:
+            actions.append("land")
+        if silu_todo:
+            actions.append("silu")  # may run after abort: a warp past its score wait still arrives
+        if drain_i < len(drain):
+            x = drain[drain_i]
+            if (stand_in_on_abort and not drain_arrived) or bars[x % nbar].done(x // nbar):
+                actions.append("drain")
+        if not actions:
+            break
+        a = actions[rng.integers(len(actions))]
+        if a == "arm":
+            x = arm_order[armed]
+            armed += 1
+            bars[x % nbar].arrive(x // nbar, tx=1)
+            in_flight.append(x)
+            if x < 3:
+                bars[x % nbar].arrive(x // nbar, n=4)
+        elif a == "mma":
+            x = arm_order[mma_next]
+            mma_next += 1
+            mma_done.add(x)
+            if x < tiles:
+                silu_todo.append(x)  # S_x computed: its SiLU tile feeds group x + 3
+        elif a == "land":
+            x = in_flight.pop(rng.integers(len(in_flight)))
+            bars[x % nbar].bytes_landed(1)
+        elif a == "silu":
+            t = silu_todo.pop(0)
+            # after a stand-in drain a late arrival may meet a phase the drain already opened
+            bars[(t + 3) % nbar].arrive((t + 3) // nbar, n=4, check_phase=not stand_in_on_abort)
+        else:
+            x = drain[drain_i]
+            if stand_in_on_abort and not drain_arrived:
+                bars[x % nbar].arrive(x // nbar, n=4, check_phase=False)  # the earlier drain's stand-ins
+                drain_arrived = True
+            else:
+                drain_i += 1  # this phase completed: its copies landed
+                drain_arrived = False
+    if not aborted:
+        assert mma_next == len(arm_order) and not in_flight
+    return step, drain, drain_i
+
+
+def test_group_barriers_hold_under_random_interleavings_and_aborts():
+    """No arrival ever meets a phase with none pending, with or without an abort, and once every
+    copy has landed a drained phase is either complete or still waits for SiLU arrivals that will
+    never come (the case the drain's time budget covers)."""
+    rng = np.random.default_rng(7)
+    for trial in range(800):
+        tiles = int(rng.integers(1, 30))
+        total, _, _ = simulate(tiles, rng)  # no abort: every group runs
+        simulate(tiles, rng, abort_at=int(rng.integers(1, total + 1)))
+
+
+def test_stand_in_arrivals_on_abort_can_meet_a_phase_with_none_pending():
+    """The earlier drain (four stand-in arrivals, then a wait) reaches an arrival on a phase with
+    no arrivals pending while bytes are outstanding in some interleavings."""
+    hit = 0
+    for trial in range(600):
+        rng = np.random.default_rng(trial)
+        tiles = int(rng.integers(4, 30))
+        total, _, _ = simulate(tiles, np.random.default_rng(trial))
+        try:
+            simulate(tiles, np.random.default_rng(trial + 1000), abort_at=int(rng.integers(1, total + 1)),
+                     stand_in_on_abort=True)
+        except AssertionError as e:
+            if "no pending arrivals" in str(e):
+                hit += 1
+    assert hit > 0
