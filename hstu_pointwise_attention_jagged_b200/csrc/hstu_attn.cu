@@ -603,7 +603,8 @@ hstu_status_t run_bwd(const void* q, const void* k, const void* v, const void* d
         cudaSuccess) {
       ds_ws = nullptr;
       cudaGetLastError();  // an allocation the pool cannot serve is not an error of the call
-    } else if (!encode_matrix(&tds, ds_ws, ds_tiles * kTileRows, kTileRows, kTileRows)) {
+    } else if ((reinterpret_cast<uintptr_t>(ds_ws) & 31u) != 0 ||  // the dS stores are 32-byte vectors
+               !encode_matrix(&tds, ds_ws, ds_tiles * kTileRows, kTileRows, kTileRows)) {
       cudaFreeAsync(ds_ws, stream);
       ds_ws = nullptr;
     }

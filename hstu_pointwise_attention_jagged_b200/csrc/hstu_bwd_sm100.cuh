@@ -165,9 +165,14 @@ __device__ __forceinline__ void bwd_grads(const uint32_t (&dp)[32], const float 
   }
   ptx::tmem_st16(t_ds, pk);
   if (g_ds != nullptr) {
-    // The same 32 values into the dS workspace for the dQ pass (written once, read by another kernel).
+    // The same 32 values into the dS workspace for the dQ pass (written once, read by another
+    // kernel): 64 bytes, 32-byte aligned, as two whole-sector stores.
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) g_ds[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+    for (int h = 0; h < 2; ++h)
+      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(g_ds + 2 * h),
+                   "r"(pk[8 * h]), "r"(pk[8 * h + 1]), "r"(pk[8 * h + 2]), "r"(pk[8 * h + 3]), "r"(pk[8 * h + 4]),
+                   "r"(pk[8 * h + 5]), "r"(pk[8 * h + 6]), "r"(pk[8 * h + 7])
+                   : "memory");
   }
 }
 
