@@ -62,7 +62,7 @@ struct BwdSchedArgs {
 // no items), then writes both lists with a counting sort over cost bins.
 __global__ void __launch_bounds__(kSchedThreads) bwd_schedule_kernel(const BwdSchedArgs a) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ int hist[kMaxCostBins];
+  __shared__ int hist[2][kMaxCostBins];
   __shared__ long long scan_scratch[2][32];
   __shared__ long long carry, carry_ds;
   __shared__ int s_L[kCachedUsers], s_U[kCachedUsers], s_ts[kCachedUsers + 1];
@@ -131,54 +131,64 @@ __global__ void __launch_bounds__(kSchedThreads) bwd_schedule_kernel(const BwdSc
     }
   };
 
-  for (int list = 0; list < 2; ++list) {
-    int4* items = list == 0 ? a.dq_items : a.kv_items;
-    for (int i = tid; i < nbins; i += kSchedThreads) hist[i] = 0;
-    __syncthreads();
-    auto cost_of = [&](int t, int L, int U) {
-      return tile_count(list == 0 ? key_tiles_of_query_tile(t, L, U) : query_tiles_of_key_tile(t, L, U));
-    };
-    for (int g = tid; g < ntiles; g += kSchedThreads) {
-      int b, t, L, U;
-      tile_of(g, b, t, L, U);
-      const int c = cost_of(t, L, U);
-      atomicAdd(&hist[c < nbins ? c : nbins - 1], a.H);
+  // Both lists in one sweep: cost histograms, one two-value scan over the bins (costlier bins
+  // first), then one scatter pass.  List 0 is the dQ list (items own a query tile), list 1 the
+  // dK/dV list (items own a key tile).
+  for (int i = tid; i < nbins; i += kSchedThreads) {
+    hist[0][i] = 0;
+    hist[1][i] = 0;
+  }
+  __syncthreads();
+  for (int g = tid; g < ntiles; g += kSchedThreads) {
+    int b, t, L, U;
+    tile_of(g, b, t, L, U);
+    const int c0 = tile_count(key_tiles_of_query_tile(t, L, U));
+    const int c1 = tile_count(query_tiles_of_key_tile(t, L, U));
+    atomicAdd(&hist[0][c0 < nbins ? c0 : nbins - 1], a.H);
+    atomicAdd(&hist[1][c1 < nbins ? c1 : nbins - 1], a.H);
+  }
+  __syncthreads();
+  const int per = cdiv(nbins, kSchedThreads);
+  long long part0 = 0, part1 = 0;
+  for (int k = 0; k < per; ++k) {
+    const int bin = nbins - 1 - (tid * per + k);
+    if (bin >= 0) {
+      part0 += hist[0][bin];
+      part1 += hist[1][bin];
     }
-    __syncthreads();
-    const int per = cdiv(nbins, kSchedThreads);
-    long long part = 0;
-    for (int k = 0; k < per; ++k) {
-      const int bin = nbins - 1 - (tid * per + k);
-      if (bin >= 0) part += hist[bin];
+  }
+  long long incl0 = part0, incl1 = part1, tot0, tot1;
+  block_inclusive_scan2(incl0, incl1, scan_scratch, tot0, tot1);
+  long long run0 = incl0 - part0, run1 = incl1 - part1;
+  for (int k = 0; k < per; ++k) {
+    const int bin = nbins - 1 - (tid * per + k);
+    if (bin >= 0) {
+      const int n0 = hist[0][bin], n1 = hist[1][bin];
+      hist[0][bin] = (int)run0;
+      hist[1][bin] = (int)run1;
+      run0 += n0;
+      run1 += n1;
     }
-    __syncthreads();
-    long long tot;
-    const long long incl = block_inclusive_scan(part, scan_scratch[0], &tot);
-    long long run = incl - part;
-    for (int k = 0; k < per; ++k) {
-      const int bin = nbins - 1 - (tid * per + k);
-      if (bin >= 0) {
-        const int n = hist[bin];
-        hist[bin] = (int)run;
-        run += n;
-      }
+  }
+  __syncthreads();
+  if (tid < 2) {
+    const long long tot = tid == 0 ? tot0 : tot1;
+    a.header[4 * tid + 0] = 0;
+    a.header[4 * tid + 1] = (int)(tot < a.max_items ? tot : a.max_items);
+    a.header[4 * tid + 2] = 0;
+    a.header[4 * tid + 3] = 0;
+  }
+  for (int g = tid; g < ntiles; g += kSchedThreads) {
+    int b, t, L, U;
+    tile_of(g, b, t, L, U);
+    const int c0 = tile_count(key_tiles_of_query_tile(t, L, U));
+    const int c1 = tile_count(query_tiles_of_key_tile(t, L, U));
+    const int pos0 = atomicAdd(&hist[0][c0 < nbins ? c0 : nbins - 1], a.H);
+    const int pos1 = atomicAdd(&hist[1][c1 < nbins ? c1 : nbins - 1], a.H);
+    for (int h = 0; h < a.H; ++h) {
+      if (pos0 + h < a.max_items) a.dq_items[pos0 + h] = make_int4(b, t, h, c0);
+      if (pos1 + h < a.max_items) a.kv_items[pos1 + h] = make_int4(b, t, h, c1);
     }
-    __syncthreads();
-    if (tid == 0) {
-      a.header[4 * list + 0] = 0;
-      a.header[4 * list + 1] = (int)(tot < a.max_items ? tot : a.max_items);
-      a.header[4 * list + 2] = 0;
-      a.header[4 * list + 3] = 0;
-    }
-    for (int g = tid; g < ntiles; g += kSchedThreads) {
-      int b, t, L, U;
-      tile_of(g, b, t, L, U);
-      const int c = cost_of(t, L, U);
-      const int pos = atomicAdd(&hist[c < nbins ? c : nbins - 1], a.H);
-      for (int h = 0; h < a.H; ++h)
-        if (pos + h < a.max_items) items[pos + h] = make_int4(b, t, h, c);
-    }
-    __syncthreads();
   }
 }
 
