@@ -318,6 +318,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       int j = 0;          // K/V loads issued
       int g = 0;          // score tiles (groups with an S) armed
       int armed_hi = 0;   // one past the highest group index armed
+      bool q_unarmed = false;  // a Q copy is on group g's barrier, whose arrival is still to come
       // V rows and heads of tiles g-3, g-2, g-1.
       int vrow0 = 0, vrow1 = 0, vrow2 = 0, vh0 = 0, vh1 = 0, vh2 = 0;
       bool ok = true;
@@ -373,20 +374,28 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             ok = false;
             break;
           }
+          // The query tile's Q goes out at once, ahead of its first K and V tiles, which wait for
+          // ring slots: its bytes join the first group's barrier without an arrival, and the
+          // producer's one arrival for that group comes with the K/V bytes below.  (Group g - 8's
+          // phase on that barrier completed before group g - 1 was armed.)
+          {
+            const uint32_t rb = bar(ctl->g_ready[g & (kGroupBars - 1)]);
+            ptx::mbar_expect_tx(rb, Cfg::kTileBytes);
+            tma_tile(&tm_q, sQ + qb * Cfg::kTileBytes, rb, w.h * D, w.q_row0);
+            ++sub;
+            q_unarmed = true;
+          }
           for (int k = 0; k < n; ++k) {
-            // Group g reads V_{g-3} (load j) and K_g (load j+1), or K_g alone for g < 3, and Q on
-            // a query tile's first tile; all of them land on the group's ready barrier.
+            // Group g reads V_{g-3} (load j) and K_g (load j+1), or K_g alone for g < 3; they and
+            // (on a query tile's first tile) Q land on the group's ready barrier.
             const bool has_v = g >= 3;
             if (!slot_free(j) || (has_v && !slot_free(j + 1))) { ok = false; break; }
             const int krow = w.kv_start + tile_at(r, k) * kTileRows;
             const uint32_t rb = bar(ctl->g_ready[g & (kGroupBars - 1)]);
-            ptx::mbar_arrive_expect_tx(rb, Cfg::kTileBytes * (1 + (has_v ? 1 : 0) + (k == 0 ? 1 : 0)));
+            ptx::mbar_arrive_expect_tx(rb, Cfg::kTileBytes * (1 + (has_v ? 1 : 0)));
             if (!has_v)  // no P.V in this group: stand in for the SiLU warps' arrivals
               for (int a = 0; a < 4; ++a) ptx::mbar_arrive(rb);
-            if (k == 0) {
-              tma_tile(&tm_q, sQ + qb * Cfg::kTileBytes, rb, w.h * D, w.q_row0);
-              ++sub;
-            }
+            q_unarmed = false;
             if (has_v) {
               tma_tile(&tm_v, sKV + (j % Cfg::kStages) * Cfg::kTileBytes, rb, vh0 * D, vrow0);
               ++j;
@@ -428,6 +437,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const uint32_t par = (uint32_t)((x / kGroupBars) & 1);
           while (!ptx::mbar_test_wait(rb, par) && ptx::globaltimer_ns() - t0 < kCopyGraceNs) {
           }
+        }
+        // A Q copy on a group that was never armed: that phase cannot complete, so the budget runs.
+        while (q_unarmed && ptx::globaltimer_ns() - t0 < kCopyGraceNs) {
         }
       }
     }

@@ -41,6 +41,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// Adds `bytes` to the transaction count the current phase waits for, without an arrival.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
 // True once the phase with parity `parity` has completed (a fresh barrier reports its
 // "preceding" phase, parity 1, as complete).  The thread may stay suspended inside the
 // instruction for at most suspend_ns (suspendTimeHint) instead of the system-dependent time.
