@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //               which CTA 1 waited on its own barrier and then arrived on CTA 0's cost one
 //               cluster-scope round trip per stage and halved the throughput.)
 //   warps 2..5  epilogue (both CTAs): its 128 rows of the accumulator, then an arrival on CTA 0's
-//               `acc_empty` (eight arrivals: four warps in each CTA).  Eight warps, two per TMEM
+//               `acc_empty` (eight arrivals: four warps in each CTA), released at CTA scope.  Eight warps, two per TMEM
 //               lane quarter, measured no faster.
 // Every wait is bounded; on a timeout the CTA records it, leaves its loops and drains, and the
 // peer's waits on it run out in turn.
@@ -462,7 +462,9 @@ __global__ void __launch_bounds__(kGemm2Threads, 1)
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(bar(ctl->acc_empty[acc]), 0));
+      // Release at CTA scope, not cluster scope: the latter held each warp until its 64 KB of C
+      // stores were visible and cost the K = 512 projection a fifth of its throughput.
+      if (lane == 0) ptx::mbar_arrive_remote(ptx::mapa_shared(bar(ctl->acc_empty[acc]), 0));
       acc ^= 1;
     }
   }

@@ -297,10 +297,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
-// Arrive (release at cluster scope) on an mbarrier given by its shared::cluster address, which
-// may be in another CTA of the cluster.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+// Arrive on an mbarrier given by its shared::cluster address, which may be in another CTA of the
+// cluster, with the default semantics (release at CTA scope).  A release at cluster scope would
+// also hold the thread until every global store it issued is visible cluster-wide; a TMEM hand-off
+// (tcgen05.wait + tcgen05.fence::before_thread_sync, then this arrival) needs none of that.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // Waits of a thread that must also see memory written by the peer CTA before its arrival.
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity, uint32_t suspend_ns) {
