@@ -73,6 +73,9 @@ struct SchedArgs {
   const int32_t* num_targets;  // [B] or null
   const int32_t* cached_len;   // [B] or null
   int32_t B, H, total_kv, total_q, max_seq_len, nbins, max_items;
+  // Users are taken in waves by their first key row (wave = row / wave_rows, at most nwaves - 1),
+  // each wave's K and V about a fixed share of L2; waves run in order, items by cost within one.
+  int32_t wave_rows, nwaves;
   int32_t* q_start;       // [B] out: first query row of each user, -1 if the user is skipped
   int32_t* block_start;    // [B+1] out: index of each user's first 128-row block among all blocks
   int4* items;            // [max_items] out: {b, pair, h, cost}, non-increasing cost
@@ -165,8 +168,12 @@ __device__ __forceinline__ int owner_of(const int32_t* block_start, int B, int g
 }
 
 // One CTA of kSchedThreads threads.  Validates every user, assigns query-row starts, and writes
-// the work items sorted by non-increasing cost (counting sort over cost bins; ties in any order).
-// The per-block passes run one thread per (user, 128-row block).
+// the work items wave by wave, each wave's items by non-increasing cost (counting sort over
+// (wave, cost) keys; ties in any order).  A wave is the users whose first key row falls in one
+// window of wave_rows rows: so the K and V tiles that the CTAs running at one time share stay in
+// L2, instead of every user's tiles being fetched again for each cost level.  A batch whose K and
+// V fit the window is one wave, ordered by cost alone.  The per-block passes run one thread per
+// (user, 128-row block).
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs a) {
   // A dependent attention kernel may start its prologue now; it waits for this grid's writes
   // (griddepcontrol.wait) before it reads anything in global memory.
@@ -176,13 +183,14 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
   __shared__ long long carry_q, carry_p;
   // Per-user values of pass 1, kept on chip for passes 2 and 4 when the batch is small enough
   // (their reads are then shared-memory latency instead of a chain of global loads).
-  __shared__ int s_L[kCachedUsers], s_U[kCachedUsers], s_c[kCachedUsers], s_q[kCachedUsers];
+  __shared__ int s_L[kCachedUsers], s_U[kCachedUsers], s_c[kCachedUsers], s_q[kCachedUsers], s_w[kCachedUsers];
   __shared__ int s_ps[kCachedUsers + 1];
   const bool cached = a.B <= kCachedUsers;
   const int tid = threadIdx.x;
   const int nbins = a.nbins;
+  const int nkeys = nbins * a.nwaves;  // <= kMaxCostBins (host)
 
-  for (int i = tid; i < nbins; i += kSchedThreads) hist[i] = 0;
+  for (int i = tid; i < nkeys; i += kSchedThreads) hist[i] = 0;
   if (tid == 0) {
     carry_q = 0;
     carry_p = 0;
@@ -231,6 +239,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
         s_c[b] = c;
         s_q[b] = ok ? (int)start_q : -1;
         s_ps[b] = (int)start_p;
+        s_w[b] = ok ? min(a.seq_offsets[b] / a.wave_rows, a.nwaves - 1) : 0;
       }
     }
     __syncthreads();
@@ -247,8 +256,9 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
     if (carry_q != a.total_q) atomicOr(a.err, kErrBadOffsets);
   }
   __syncthreads();
-  // Cost of block g (and its user), from shared memory when cached.
-  auto block_of = [&](int g, int& b, int& pr, int& cost) {
+  // Cost of block g (and its user), from shared memory when cached; `key` orders the items: its
+  // wave first, then non-increasing cost.
+  auto block_of = [&](int g, int& b, int& pr, int& cost, int& key) {
     b = owner_of(cached ? s_ps : a.block_start, a.B, g);
     if ((cached ? s_q[b] : a.q_start[b]) < 0) return false;
     const int L = cached ? s_L[b] : a.seq_offsets[b + 1] - a.seq_offsets[b];
@@ -257,33 +267,35 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
     pr = g - (cached ? s_ps[b] : a.block_start[b]);
     const int rows = (L - c) - pr * kItemRows;
     cost = item_cost(c + pr * kItemRows, rows < kItemRows ? rows : kItemRows, U);
+    const int wave = cached ? s_w[b] : min(a.seq_offsets[b] / a.wave_rows, a.nwaves - 1);
+    key = wave * nbins + (nbins - 1 - (cost < nbins ? cost : nbins - 1));
     return true;
   };
 
-  // Pass 2: cost histogram, one thread per block.
+  // Pass 2: key histogram, one thread per block.
   for (int g = tid; g < nblocks_total; g += kSchedThreads) {
-    int b, pr, cost;
-    if (!block_of(g, b, pr, cost)) continue;
-    atomicAdd(&hist[cost < nbins ? cost : nbins - 1], a.H);
+    int b, pr, cost, key;
+    if (!block_of(g, b, pr, cost, key)) continue;
+    atomicAdd(&hist[key], a.H);
   }
   __syncthreads();
 
-  // Pass 3: bin start = number of items in strictly costlier bins (descending order).
-  const int per = cdiv(nbins, kSchedThreads);
+  // Pass 3: key start = number of items with smaller keys.
+  const int per = cdiv(nkeys, kSchedThreads);
   long long part = 0;
   for (int k = 0; k < per; ++k) {
-    const int bin = nbins - 1 - (tid * per + k);
-    if (bin >= 0) part += hist[bin];
+    const int key = tid * per + k;
+    if (key < nkeys) part += hist[key];
   }
   __syncthreads();
   long long tot;
   const long long incl = block_inclusive_scan(part, scan_scratch[0], &tot);
   long long run = incl - part;
   for (int k = 0; k < per; ++k) {
-    const int bin = nbins - 1 - (tid * per + k);
-    if (bin >= 0) {
-      const int n = hist[bin];
-      hist[bin] = (int)run;
+    const int key = tid * per + k;
+    if (key < nkeys) {
+      const int n = hist[key];
+      hist[key] = (int)run;
       run += n;
     }
   }
@@ -294,11 +306,11 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const SchedArgs
     *a.done_counter = 0;
   }
 
-  // Pass 4: scatter the items into their bins, one thread per block.
+  // Pass 4: scatter the items into their keys' ranges, one thread per block.
   for (int g = tid; g < nblocks_total; g += kSchedThreads) {
-    int b, pr, cost;
-    if (!block_of(g, b, pr, cost)) continue;
-    const int pos = atomicAdd(&hist[cost < nbins ? cost : nbins - 1], a.H);
+    int b, pr, cost, key;
+    if (!block_of(g, b, pr, cost, key)) continue;
+    const int pos = atomicAdd(&hist[key], a.H);
     for (int h = 0; h < a.H; ++h)
       if (pos + h < a.max_items) a.items[pos + h] = make_int4(b, pr, h, cost);
   }

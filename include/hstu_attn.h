@@ -160,9 +160,13 @@ hstu_status_t hstu_attn_fwd_rab(const void* q, const void* k, const void* v,
  *     q_start[B]         first query row of each user (-1: user skipped), padded to 16 bytes
  *     block_start[B+1]   index of each user's first 128-row block, padded to 16 bytes
  *     items[cap][4]      {b, block, h, cost}, cap = H * (total_q / 128 + B); the first
- *                        num_items entries are valid, in non-increasing cost order.  `block` is
- *                        a block of 128 query rows of user b; `cost` is the number of 128x128
- *                        score tiles the block computes (fully masked tiles are not counted).
+ *                        num_items entries are valid.  `block` is a block of 128 query rows of
+ *                        user b; `cost` is the number of 128x128 score tiles the block computes
+ *                        (fully masked tiles are not counted).  Order: users are taken in waves
+ *                        by their first key row, floor(seq_offsets[b] / W) with
+ *                        W = 64 MiB / (512 * H) rows (the rows whose K and V fill about half of
+ *                        L2 at d = 128), and items go by wave, then by non-increasing cost; a
+ *                        batch of fewer than W rows is in non-increasing cost order.
  *
  * hstu_attn_plan — validates the offsets on the device and writes the plan.
  *   seq_offsets, num_targets, cached_len, B, H, total_kv, total_q, max_seq_len: as in
