@@ -50,6 +50,9 @@ struct BwdSchedArgs {
   const int32_t* seq_offsets;  // [B+1]
   const int32_t* num_targets;  // [B] or null
   int32_t B, H, total, max_seq_len, nbins, max_items;
+  // Waves of users by first row (wave = row / wave_rows, at most nwaves - 1): items go by wave,
+  // then by non-increasing cost, so the tiles streamed at one time stay in L2.
+  int32_t wave_rows, nwaves;
   int32_t* header;      // [8] out: {dq counter, dq items, dq done, 0, kv counter, kv items, kv done, 0}
   int32_t* tile_start;  // [B+1] out: index of each user's first 128-row tile among all tiles
   long long* ds_base;   // [B+1] out: index of each user's first dS tile (all heads); may be null
@@ -59,16 +62,17 @@ struct BwdSchedArgs {
 };
 
 // One CTA of kSchedThreads threads: validates every user (a bad user sets kErrBadOffsets and gets
-// no items), then writes both lists with a counting sort over cost bins.
+// no items), then writes both lists with a counting sort over (wave, cost) keys.
 __global__ void __launch_bounds__(kSchedThreads) bwd_schedule_kernel(const BwdSchedArgs a) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ int hist[2][kMaxCostBins];
   __shared__ long long scan_scratch[2][32];
   __shared__ long long carry, carry_ds;
-  __shared__ int s_L[kCachedUsers], s_U[kCachedUsers], s_ts[kCachedUsers + 1];
+  __shared__ int s_L[kCachedUsers], s_U[kCachedUsers], s_ts[kCachedUsers + 1], s_w[kCachedUsers];
   const bool cached = a.B <= kCachedUsers;
   const int tid = threadIdx.x;
   const int nbins = a.nbins;
+  const int nkeys = nbins * a.nwaves;  // <= kMaxCostBins (host)
   if (tid == 0) carry = carry_ds = 0;
   __syncthreads();
 
@@ -100,6 +104,7 @@ __global__ void __launch_bounds__(kSchedThreads) bwd_schedule_kernel(const BwdSc
         s_L[b] = L;
         s_U[b] = U;
         s_ts[b] = (int)start;
+        s_w[b] = min(a.seq_offsets[b] / a.wave_rows, a.nwaves - 1);
       }
     }
     __syncthreads();
@@ -119,53 +124,56 @@ __global__ void __launch_bounds__(kSchedThreads) bwd_schedule_kernel(const BwdSc
 
   // Tile g: its user, its index within the user, and the user's L and U.  Users skipped in
   // pass 1 own no tiles.
-  auto tile_of = [&](int g, int& b, int& t, int& L, int& U) {
+  auto tile_of = [&](int g, int& b, int& t, int& L, int& U, int& wave) {
     b = owner_of(cached ? s_ts : a.tile_start, a.B, g);
     t = g - (cached ? s_ts[b] : a.tile_start[b]);
     if (cached) {
       L = s_L[b];
       U = s_U[b];
+      wave = s_w[b];
     } else {
       L = a.seq_offsets[b + 1] - a.seq_offsets[b];
       U = L - (a.num_targets ? a.num_targets[b] : 0);
+      wave = min(a.seq_offsets[b] / a.wave_rows, a.nwaves - 1);
     }
   };
+  auto key_of = [&](int wave, int c) { return wave * nbins + (nbins - 1 - (c < nbins ? c : nbins - 1)); };
 
   // Both lists in one sweep: cost histograms, one two-value scan over the bins (costlier bins
   // first), then one scatter pass.  List 0 is the dQ list (items own a query tile), list 1 the
   // dK/dV list (items own a key tile).
-  for (int i = tid; i < nbins; i += kSchedThreads) {
+  for (int i = tid; i < nkeys; i += kSchedThreads) {
     hist[0][i] = 0;
     hist[1][i] = 0;
   }
   __syncthreads();
   for (int g = tid; g < ntiles; g += kSchedThreads) {
-    int b, t, L, U;
-    tile_of(g, b, t, L, U);
+    int b, t, L, U, wave;
+    tile_of(g, b, t, L, U, wave);
     const int c0 = tile_count(key_tiles_of_query_tile(t, L, U));
     const int c1 = tile_count(query_tiles_of_key_tile(t, L, U));
-    atomicAdd(&hist[0][c0 < nbins ? c0 : nbins - 1], a.H);
-    atomicAdd(&hist[1][c1 < nbins ? c1 : nbins - 1], a.H);
+    atomicAdd(&hist[0][key_of(wave, c0)], a.H);
+    atomicAdd(&hist[1][key_of(wave, c1)], a.H);
   }
   __syncthreads();
-  const int per = cdiv(nbins, kSchedThreads);
+  const int per = cdiv(nkeys, kSchedThreads);
   long long part0 = 0, part1 = 0;
   for (int k = 0; k < per; ++k) {
-    const int bin = nbins - 1 - (tid * per + k);
-    if (bin >= 0) {
-      part0 += hist[0][bin];
-      part1 += hist[1][bin];
+    const int key = tid * per + k;
+    if (key < nkeys) {
+      part0 += hist[0][key];
+      part1 += hist[1][key];
     }
   }
   long long incl0 = part0, incl1 = part1, tot0, tot1;
   block_inclusive_scan2(incl0, incl1, scan_scratch, tot0, tot1);
   long long run0 = incl0 - part0, run1 = incl1 - part1;
   for (int k = 0; k < per; ++k) {
-    const int bin = nbins - 1 - (tid * per + k);
-    if (bin >= 0) {
-      const int n0 = hist[0][bin], n1 = hist[1][bin];
-      hist[0][bin] = (int)run0;
-      hist[1][bin] = (int)run1;
+    const int key = tid * per + k;
+    if (key < nkeys) {
+      const int n0 = hist[0][key], n1 = hist[1][key];
+      hist[0][key] = (int)run0;
+      hist[1][key] = (int)run1;
       run0 += n0;
       run1 += n1;
     }
@@ -179,12 +187,12 @@ __global__ void __launch_bounds__(kSchedThreads) bwd_schedule_kernel(const BwdSc
     a.header[4 * tid + 3] = 0;
   }
   for (int g = tid; g < ntiles; g += kSchedThreads) {
-    int b, t, L, U;
-    tile_of(g, b, t, L, U);
+    int b, t, L, U, wave;
+    tile_of(g, b, t, L, U, wave);
     const int c0 = tile_count(key_tiles_of_query_tile(t, L, U));
     const int c1 = tile_count(query_tiles_of_key_tile(t, L, U));
-    const int pos0 = atomicAdd(&hist[0][c0 < nbins ? c0 : nbins - 1], a.H);
-    const int pos1 = atomicAdd(&hist[1][c1 < nbins ? c1 : nbins - 1], a.H);
+    const int pos0 = atomicAdd(&hist[0][key_of(wave, c0)], a.H);
+    const int pos1 = atomicAdd(&hist[1][key_of(wave, c1)], a.H);
     for (int h = 0; h < a.H; ++h) {
       if (pos0 + h < a.max_items) a.dq_items[pos0 + h] = make_int4(b, t, h, c0);
       if (pos1 + h < a.max_items) a.kv_items[pos1 + h] = make_int4(b, t, h, c1);

@@ -621,6 +621,10 @@ hstu_status_t run_bwd(const void* q, const void* k, const void* v, const void* d
   a.total = total;
   a.max_seq_len = max_seq_len;
   a.nbins = cost_bins(max_seq_len);
+  // Waves of users whose streamed pairs (Q and dO, or K and V: 512 bytes per row and head at
+  // d = 128) take about a quarter of L2.
+  a.wave_rows = static_cast<int32_t>((32ll << 20) / (512ll * H) > 0 ? (32ll << 20) / (512ll * H) : 1);
+  a.nwaves = kMaxCostBins / a.nbins > 0 ? kMaxCostBins / a.nbins : 1;
   a.max_items = static_cast<int32_t>(cap);
   a.header = header;
   a.tile_start = tile_start;
