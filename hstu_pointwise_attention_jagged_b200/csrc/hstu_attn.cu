@@ -241,9 +241,9 @@ cudaError_t launch_plan(const int32_t* seq_offsets, const int32_t* num_targets, 
   a.max_seq_len = max_seq_len;
   a.nbins = cost_bins(max_seq_len);
   a.max_items = static_cast<int32_t>(capacity(B, H, total_q));
-  // Waves of users whose K and V (sized for d = 128: 512 bytes per row and head) take about half
-  // of the 126 MB L2; as many waves as the key space allows.
-  a.wave_rows = static_cast<int32_t>((64ll << 20) / (512ll * H) > 0 ? (64ll << 20) / (512ll * H) : 1);
+  // Waves of users whose K and V (sized for d = 128: 512 bytes per row and head) take about a
+  // quarter of the 126 MB L2; as many waves as the key space allows.
+  a.wave_rows = static_cast<int32_t>((32ll << 20) / (512ll * H) > 0 ? (32ll << 20) / (512ll * H) : 1);
   a.nwaves = kMaxCostBins / a.nbins > 0 ? kMaxCostBins / a.nbins : 1;
   a.q_start = w.q_start;
   a.block_start = w.block_start;

@@ -164,8 +164,8 @@ hstu_status_t hstu_attn_fwd_rab(const void* q, const void* k, const void* v,
  *                        user b; `cost` is the number of 128x128 score tiles the block computes
  *                        (fully masked tiles are not counted).  Order: users are taken in waves
  *                        by their first key row, floor(seq_offsets[b] / W) with
- *                        W = 64 MiB / (512 * H) rows (the rows whose K and V fill about half of
- *                        L2 at d = 128), and items go by wave, then by non-increasing cost; a
+ *                        W = 32 MiB / (512 * H) rows (the rows whose K and V fill about a quarter
+ *                        of L2 at d = 128), and items go by wave, then by non-increasing cost; a
  *                        batch of fewer than W rows is in non-increasing cost order.
  *
  * hstu_attn_plan — validates the offsets on the device and writes the plan.

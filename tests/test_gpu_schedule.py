@@ -1,7 +1,7 @@
 """GPU: the device-built work plan, bit-exact against an enumeration written from the mask's
 definition (integer work: compared exactly; the order of equal keys is free, so the multiset is
 compared and the order checked).  The plan takes users in waves by their first key row, each wave's K
-and V about 64 MB at d = 128 (64 MiB / (512 bytes x H) rows), and orders items by wave, then by
+and V about 32 MB at d = 128 (32 MiB / (512 bytes x H) rows), and orders items by wave, then by
 non-increasing cost; a batch within one window is ordered by cost alone."""
 import math
 
@@ -71,7 +71,7 @@ def test_schedule_matches_definition(case):
     max_len = int(L.max())
     nbins = min(2 * (max_len // 128 + 3) + 1, 4096)
     nwaves = max(4096 // nbins, 1)
-    wave_rows = max((64 << 20) // (512 * H), 1)
+    wave_rows = max((32 << 20) // (512 * H), 1)
     keys = [(min(int(off[g[0]]) // wave_rows, nwaves - 1), -g[3]) for g in got]
     assert all(keys[i] <= keys[i + 1] for i in range(len(keys) - 1))
     assert binding.hstu_attn_get_error() == 0
