@@ -204,6 +204,15 @@ int cost_bins(int32_t max_seq_len) {
   return static_cast<int>(n < kMaxCostBins ? n : kMaxCostBins);
 }
 
+// Waves a plan's keys need: those the batch's rows can reach, no more than the key space holds (the
+// plan kernels clear and scan waves x cost bins keys).
+int plan_waves(int64_t rows, int32_t wave_rows, int32_t nbins) {
+  const int64_t need = rows > 0 ? (rows + wave_rows - 1) / wave_rows : 1;
+  const int64_t fit = nbins > 0 ? kMaxCostBins / nbins : 1;
+  const int64_t n = need < fit ? need : fit;
+  return static_cast<int>(n > 0 ? n : 1);
+}
+
 // Scalar checks shared by every entry point.  Returns HSTU_OK or the status to report.
 hstu_status_t check_sizes(int32_t B, int32_t H, int32_t total_kv, int32_t total_q) {
   if (B < 0 || H < 1 || total_kv < 0 || total_q < 0 || total_q > total_kv) return HSTU_ERR_INVALID_ARGUMENT;
@@ -244,7 +253,7 @@ cudaError_t launch_plan(const int32_t* seq_offsets, const int32_t* num_targets, 
   // Waves of users whose K and V (sized for d = 128: 512 bytes per row and head) take about a
   // quarter of the 126 MB L2; as many waves as the key space allows.
   a.wave_rows = static_cast<int32_t>((32ll << 20) / (512ll * H) > 0 ? (32ll << 20) / (512ll * H) : 1);
-  a.nwaves = kMaxCostBins / a.nbins > 0 ? kMaxCostBins / a.nbins : 1;
+  a.nwaves = plan_waves(total_kv, a.wave_rows, a.nbins);
   a.q_start = w.q_start;
   a.block_start = w.block_start;
   a.items = w.items;
@@ -624,7 +633,7 @@ hstu_status_t run_bwd(const void* q, const void* k, const void* v, const void* d
   // Waves of users whose streamed pairs (Q and dO, or K and V: 512 bytes per row and head at
   // d = 128) take about a quarter of L2.
   a.wave_rows = static_cast<int32_t>((32ll << 20) / (512ll * H) > 0 ? (32ll << 20) / (512ll * H) : 1);
-  a.nwaves = kMaxCostBins / a.nbins > 0 ? kMaxCostBins / a.nbins : 1;
+  a.nwaves = plan_waves(total, a.wave_rows, a.nbins);
   a.max_items = static_cast<int32_t>(cap);
   a.header = header;
   a.tile_start = tile_start;

@@ -70,8 +70,8 @@ def test_schedule_matches_definition(case):
     assert sorted(got) == sorted(exp)
     max_len = int(L.max())
     nbins = min(2 * (max_len // 128 + 3) + 1, 4096)
-    nwaves = max(4096 // nbins, 1)
     wave_rows = max((32 << 20) // (512 * H), 1)
+    nwaves = max(min(4096 // nbins, -(-total_kv // wave_rows)), 1)
     keys = [(min(int(off[g[0]]) // wave_rows, nwaves - 1), -g[3]) for g in got]
     assert all(keys[i] <= keys[i + 1] for i in range(len(keys) - 1))
     assert binding.hstu_attn_get_error() == 0
