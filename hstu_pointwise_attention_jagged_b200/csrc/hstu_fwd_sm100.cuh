@@ -224,9 +224,9 @@ __device__ __forceinline__ void load_bias(float (&b)[32], const float* rab_row, 
   }
 }
 
-template <int kChunk, bool kRab>
+template <int kChunk, bool kRab, bool kMasked>
 __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t taddr_s, float half_alpha,
-                                           bool full, int lim, int self, const float (&bias)[32]) {
+                                           int lim, int self, const float (&bias)[32]) {
   uint32_t pk[16];
   // Columns are taken in pairs on the two-wide FMA pipe: h = s * alpha/2 and p = h * tanh(h) + h,
   // bit-identical to the scalar forms.
@@ -242,7 +242,7 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t tad
       p0 += bias[2 * e];
       p1 += bias[2 * e + 1];
     }
-    if (!full) {
+    if constexpr (kMasked) {
       const int c0 = kChunk * 32 + 2 * e;
       p0 = (c0 < lim || c0 == self) ? p0 : 0.0f;
       p1 = (c0 + 1 < lim || c0 + 1 == self) ? p1 : 0.0f;
@@ -250,6 +250,34 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&r)[32], uint32_t tad
     pk[e] = pack_bf16x2(p0, p1);
   }
   ptx::tmem_st16(taddr_s + kChunk * 16, pk);
+}
+
+// The SiLU of one score tile for this thread's row: four 32-column chunks, each read from TMEM,
+// transformed and written back as packed bf16 over the first 64 columns.  A tile that lies inside
+// every one of its rows' visible ranges takes the kMasked = false form, which has no per-column
+// tests at all; only tiles that cross the diagonal or the history edge take the masked form.
+// Chunks are loaded one at a time: the registers a second buffer would take keep the SiLU free of
+// spills, and the other SiLU warps on the scheduler cover the load latency.  With kRab, the next
+// chunk's biases are loaded as soon as the previous chunk is done.
+template <bool kMasked, bool kRab>
+__device__ __forceinline__ void silu_tile(uint32_t taddr_s, float half_alpha, int lim, int self, float (&bias)[32],
+                                          const float* rab_row, int rel0, int rab_max) {
+  uint32_t ra[32];
+  ptx::tmem_ld32(taddr_s + 0, ra);
+  ptx::tmem_ld_wait(ra);
+  silu_chunk<0, kRab, kMasked>(ra, taddr_s, half_alpha, lim, self, bias);
+  if constexpr (kRab) load_bias<1>(bias, rab_row, rel0, rab_max);
+  ptx::tmem_ld32(taddr_s + 32, ra);
+  ptx::tmem_ld_wait(ra);
+  silu_chunk<1, kRab, kMasked>(ra, taddr_s, half_alpha, lim, self, bias);
+  if constexpr (kRab) load_bias<2>(bias, rab_row, rel0, rab_max);
+  ptx::tmem_ld32(taddr_s + 64, ra);
+  ptx::tmem_ld_wait(ra);
+  silu_chunk<2, kRab, kMasked>(ra, taddr_s, half_alpha, lim, self, bias);
+  if constexpr (kRab) load_bias<3>(bias, rab_row, rel0, rab_max);
+  ptx::tmem_ld32(taddr_s + 96, ra);
+  ptx::tmem_ld_wait(ra);
+  silu_chunk<3, kRab, kMasked>(ra, taddr_s, half_alpha, lim, self, bias);
 }
 
 // Loads run K_0 K_1 K_2 | V_0 K_3 | V_1 K_4 | ... in the order the MMA warp consumes them, so load
@@ -601,25 +629,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const int lim = lim_abs - j0;
           const int self = i_pos - j0;
           const int rel0 = i_pos - j0;
-          // 32-column chunks, one at a time: the registers a second buffer would take keep the
-          // SiLU free of spills, and the other SiLU warps on the scheduler cover the load latency.
-          // With kRab, the next chunk's biases are loaded as soon as the previous chunk is done.
-          uint32_t ra[32];
-          ptx::tmem_ld32(taddr_s + 0, ra);
-          ptx::tmem_ld_wait(ra);
-          silu_chunk<0, kRab>(ra, taddr_s, half_alpha, full, lim, self, bias);
-          if constexpr (kRab) load_bias<1>(bias, rab_row, rel0, rab_max);
-          ptx::tmem_ld32(taddr_s + 32, ra);
-          ptx::tmem_ld_wait(ra);
-          silu_chunk<1, kRab>(ra, taddr_s, half_alpha, full, lim, self, bias);
-          if constexpr (kRab) load_bias<2>(bias, rab_row, rel0, rab_max);
-          ptx::tmem_ld32(taddr_s + 64, ra);
-          ptx::tmem_ld_wait(ra);
-          silu_chunk<2, kRab>(ra, taddr_s, half_alpha, full, lim, self, bias);
-          if constexpr (kRab) load_bias<3>(bias, rab_row, rel0, rab_max);
-          ptx::tmem_ld32(taddr_s + 96, ra);
-          ptx::tmem_ld_wait(ra);
-          silu_chunk<3, kRab>(ra, taddr_s, half_alpha, full, lim, self, bias);
+          // `full` is the same for every row of the tile, so the warp takes one branch.
+          if (full) {
+            silu_tile<false, kRab>(taddr_s, half_alpha, lim, self, bias, rab_row, rel0, rab_max);
+          } else {
+            silu_tile<true, kRab>(taddr_s, half_alpha, lim, self, bias, rab_row, rel0, rab_max);
+          }
           ptx::tmem_st_wait();
           ptx::tc_fence_before();
           __syncwarp();
