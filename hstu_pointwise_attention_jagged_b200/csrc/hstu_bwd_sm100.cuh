@@ -113,10 +113,11 @@ __device__ __forceinline__ BwdWork read_bwd_slot(const volatile int32_t* s) {
 // SiLU factor m = (1 + t)(1 + h - h t) of every column, kept in registers for the second half, and
 // (dK/dV) P = h (1 + t), packed as bf16 pairs into 16 TMEM columns.  The visible columns are
 // [lo, hi) plus `self` (relative to the chunk's first column); P is an exact zero elsewhere.
-// Columns go in pairs on the two-wide FMA pipe.
-template <bool kDQ>
+// Columns go in pairs on the two-wide FMA pipe.  kMasked = false is the form for a warp whose 32
+// rows see all 64 columns: it carries no per-column tests.
+template <bool kDQ, bool kMasked>
 __device__ __forceinline__ void bwd_scores(const uint32_t (&s)[32], float (&m)[32], uint32_t t_p, float half_alpha,
-                                           bool full, int lo, int hi, int self) {
+                                           int lo, int hi, int self) {
   uint32_t pk_p[16];
   const uint64_t ha2 = ptx::f32x2(half_alpha, half_alpha);
   const uint64_t one2 = ptx::f32x2(1.0f, 1.0f);
@@ -134,7 +135,7 @@ __device__ __forceinline__ void bwd_scores(const uint32_t (&s)[32], float (&m)[3
     if constexpr (!kDQ) {
       float p0, p1;
       ptx::f32x2_split(ptx::mul_f32x2(h2, a2), p0, p1);
-      if (!full) {
+      if constexpr (kMasked) {
         p0 = ((c >= lo && c < hi) || c == self) ? p0 : 0.0f;
         p1 = ((c + 1 >= lo && c + 1 < hi) || c + 1 == self) ? p1 : 0.0f;
       }
@@ -146,8 +147,9 @@ __device__ __forceinline__ void bwd_scores(const uint32_t (&s)[32], float (&m)[3
 
 // Second half: dS = (dP ds_scale) m, an exact zero outside the visible columns, packed as bf16
 // pairs into 16 TMEM columns.
+template <bool kMasked>
 __device__ __forceinline__ void bwd_grads(const uint32_t (&dp)[32], const float (&m)[32], uint32_t t_ds,
-                                          float ds_scale, bool full, int lo, int hi, int self, uint4* g_ds) {
+                                          float ds_scale, int lo, int hi, int self, uint4* g_ds) {
   uint32_t pk[16];
   const uint64_t sc2 = ptx::f32x2(ds_scale, ds_scale);
 #pragma unroll
@@ -157,7 +159,7 @@ __device__ __forceinline__ void bwd_grads(const uint32_t (&dp)[32], const float 
     ptx::f32x2_split(ptx::mul_f32x2(ptx::mul_f32x2(ptx::f32x2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), sc2),
                                     ptx::f32x2(m[c], m[c + 1])),
                      d0, d1);
-    if (!full) {
+    if constexpr (kMasked) {
       d0 = ((c >= lo && c < hi) || c == self) ? d0 : 0.0f;
       d1 = ((c + 1 >= lo && c + 1 < hi) || c + 1 == self) ? d1 : 0.0f;
     }
@@ -471,6 +473,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           self = -1;
           full = (lo <= 0) && (hi >= 64);
         }
+        // The mask-free forms run only when every row of the warp sees all 64 columns, so the warp
+        // takes one branch.
+        full = __all_sync(0xffffffffu, full);
         // First half: S -> the SiLU factors (registers) and, for dK/dV, P over S.  Then S is released.
         float m[2][32];
 #pragma unroll
@@ -478,7 +483,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t rs[32];
           ptx::tmem_ld32(t_s + 32 * k, rs);
           ptx::tmem_ld_wait(rs);
-          bwd_scores<kDQ>(rs, m[k], t_s + 16 * k, p.half_alpha, full, lo - 32 * k, hi - 32 * k, self - 32 * k);
+          if (full)
+            bwd_scores<kDQ, false>(rs, m[k], t_s + 16 * k, p.half_alpha, lo - 32 * k, hi - 32 * k, self - 32 * k);
+          else
+            bwd_scores<kDQ, true>(rs, m[k], t_s + 16 * k, p.half_alpha, lo - 32 * k, hi - 32 * k, self - 32 * k);
         }
         if constexpr (!kDQ) ptx::tmem_st_wait();
         ptx::tc_fence_before();
@@ -506,8 +514,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t rd[32];
           ptx::tmem_ld32(t_dp + 32 * k, rd);
           ptx::tmem_ld_wait(rd);
-          bwd_grads(rd, m[k], t_dp + 16 * k, p.ds_scale, full, lo - 32 * k, hi - 32 * k, self - 32 * k,
-                    g_ds ? g_ds + 4 * k : nullptr);
+          if (full)
+            bwd_grads<false>(rd, m[k], t_dp + 16 * k, p.ds_scale, lo - 32 * k, hi - 32 * k, self - 32 * k,
+                             g_ds ? g_ds + 4 * k : nullptr);
+          else
+            bwd_grads<true>(rd, m[k], t_dp + 16 * k, p.ds_scale, lo - 32 * k, hi - 32 * k, self - 32 * k,
+                            g_ds ? g_ds + 4 * k : nullptr);
         }
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
