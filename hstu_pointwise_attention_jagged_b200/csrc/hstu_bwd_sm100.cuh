@@ -129,12 +129,13 @@ __device__ __forceinline__ void bwd_scores(const uint32_t (&s)[32], float (&m)[3
     float h0, h1;
     ptx::f32x2_split(h2, h0, h1);
     const uint64_t t2 = ptx::f32x2(ptx::tanh_approx(h0), ptx::tanh_approx(h1));
-    const uint64_t a2 = ptx::fma_f32x2(t2, one2, one2);                                          // 1 + t
-    const uint64_t w2 = ptx::fma_f32x2(ptx::fma_f32x2(ptx::mul_f32x2(h2, neg2), t2, h2), one2, one2);  // 1 + h - h t
-    ptx::f32x2_split(ptx::mul_f32x2(a2, w2), m[c], m[c + 1]);
+    const uint64_t a2 = ptx::fma_f32x2(t2, one2, one2);  // 1 + t
+    const uint64_t p2 = ptx::mul_f32x2(h2, a2);          // p = h (1 + t)
+    // m = (1 + t)(1 + h - h t) = (1 + t) + p (1 - t)
+    ptx::f32x2_split(ptx::fma_f32x2(p2, ptx::fma_f32x2(t2, neg2, one2), a2), m[c], m[c + 1]);
     if constexpr (!kDQ) {
       float p0, p1;
-      ptx::f32x2_split(ptx::mul_f32x2(h2, a2), p0, p1);
+      ptx::f32x2_split(p2, p0, p1);
       if constexpr (kMasked) {
         p0 = ((c >= lo && c < hi) || c == self) ? p0 : 0.0f;
         p1 = ((c + 1 >= lo && c + 1 < hi) || c + 1 == self) ? p1 : 0.0f;
