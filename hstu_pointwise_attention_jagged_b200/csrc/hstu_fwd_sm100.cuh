@@ -5,9 +5,10 @@
 // from a cost-ordered list through an atomic counter.  Every role walks the same global sequence
 // of score tiles g = 0, 1, 2, ... over the CTA's query tiles and their visible key tiles.
 //
-//   warp 8       producer: fetches the next item, TMA-loads each query tile's Q into one of two
-//                buffers and the K and V tiles into a ring of shared-memory slots, in the order
-//                the tensor core consumes them: K_0 K_1 K_2 V_0 K_3 V_1 K_4 ... (V_{g-3}, K_g).
+//   warp 8       producer: fetches the next item, TMA-loads each query tile's Q into its buffer
+//                (one of two at d <= 64) and the K and V tiles into a ring of shared-memory
+//                slots, in the order the tensor core consumes them: K_0 K_1 K_2 V_0 K_3 V_1 K_4
+//                ... (V_{g-3}, K_g).
 //   warp 9       MMA issuer (lane 0 issues every tcgen05 instruction).  Group g is
 //                O += P_{g-3} V_{g-3}  (TS form, P read from TMEM), then S_g = Q K_g^T into score
 //                buffer g mod 3 (SS form), then one commit.  Three score buffers give the SiLU of
@@ -61,9 +62,12 @@ struct FwdCfg {
   static constexpr int kTileBytes = kBlocks * kBlockBytes;  // 128 rows x D bf16
   static constexpr uint32_t kSwizzle = (kRowBytes == 128) ? 2u : 4u;  // UMMA layout code
   static constexpr int kKStepsPerBlock = kBlockElems / 16;
-  static constexpr int kQBufs = 2;
-  // K/V ring slots: as many as fit beside the two Q buffers in 227 KB.
-  static constexpr int kStages = (D == 128) ? 5 : 10;
+  // Q buffers and K/V ring slots in 227 KB.  At d = 128 one Q buffer and six slots: a K or V copy
+  // from L2 takes longer than a group of MMAs, so the sixth slot, which lets the producer run a whole
+  // group further ahead, is worth more than loading the next query tile's Q early.  At d <= 64 two
+  // Q buffers and ten slots fit.
+  static constexpr int kQBufs = (D == 128) ? 1 : 2;
+  static constexpr int kStages = (D == 128) ? 6 : 10;
   static constexpr int kSBufs = 3;
   // The producer reuses a ring slot after waiting on the score commit of the group that consumed
   // the slot's previous tile.  That commit rotates over kSCommits barriers, so the wait is
@@ -396,8 +400,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         {
           const TileRange r = key_tiles(w.pos0, w.pos0 + w.nrows, w.U);
           const int n = tile_count(r);
-          const int qb = sub & 1;
-          if (!wait_bounded(bar(ctl->q_empty[qb]), (uint32_t)(((sub >> 1) & 1) ^ 1), abort_flag, p.err,
+          const int qb = sub % Cfg::kQBufs;
+          if (!wait_bounded(bar(ctl->q_empty[qb]), (uint32_t)(((sub / Cfg::kQBufs) & 1) ^ 1), abort_flag, p.err,
                             p.wait_limit_ns)) {
             ok = false;
             break;
@@ -535,7 +539,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       {
         const TileRange r = key_tiles(w.pos0, w.pos0 + w.nrows, w.U);
         const int n = tile_count(r);
-        const int qb = sub & 1;
+        const int qb = sub % Cfg::kQBufs;
         const uint64_t dq = dq0 + ((qb * Cfg::kTileBytes) >> 4);
         for (int k = 0; k < n; ++k) {
           // Group g: once its tiles and P_{g-3} are in, the P.V of tile g-3, then the scores of

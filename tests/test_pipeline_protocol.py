@@ -11,7 +11,7 @@ arrive on one of kGroupBars ready barriers.
 This module restates those rules in Python and replays them on random sequences of tile counts, to
 show that (1) group_of_load names the group that really consumed each load, (2) a slot is never
 reused before its previous tile was consumed, (3) no parity wait can see a barrier two phases
-ahead, for the ring depths the kernel uses (5 slots at d = 128, 10 at d <= 64), and (4) the
+ahead, for the ring depths the kernel uses (6 slots at d = 128, 10 at d <= 64), and (4) the
 constraint kStages <= 2 kSCommits - 2 stated beside the kernel's configuration is the exact limit.
 An event-level model of the group barriers then replays random interleavings of the roles, with
 and without an abort, to show that no arrival ever lands on a phase with no pending arrivals, and
@@ -72,7 +72,7 @@ def replay(tiles, stages):
     return True
 
 
-@pytest.mark.parametrize("stages", [5, 10])
+@pytest.mark.parametrize("stages", [5, 6, 10])
 def test_ring_rules_hold_for_random_streams(stages):
     rng = np.random.default_rng(100 + stages)
     for tiles in list(range(1, 40)) + list(rng.integers(40, 400, 20)):
