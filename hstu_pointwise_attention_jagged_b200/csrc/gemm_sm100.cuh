@@ -98,6 +98,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
+  // Launched as a programmatic dependent: A may come from the previous kernel, and C may be memory
+  // it still reads, so nothing global is touched before that kernel has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const int ntiles = p.tiles_m * p.tiles_n;
   const int kblocks = (p.K + kGemmBK - 1) / kGemmBK;
@@ -331,6 +334,9 @@ __global__ void __launch_bounds__(kGemm2Threads, 1)
   ptx::cluster_sync();  // the peer's barriers are initialised before anything arrives on them
   ptx::tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
+  // Launched as a programmatic dependent: A may come from the previous kernel, and C may be memory
+  // it still reads, so nothing global is touched before that kernel has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const int ntiles = p.tiles_m * p.tiles_n;
   const int kblocks = (p.K + kGemmBK - 1) / kGemmBK;

@@ -366,8 +366,20 @@ hstu_status_t launch_gemm_1sm(DeviceState* st, const void* a, const void* w, voi
   const int64_t ntiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
   if (ntiles > INT_MAX) return HSTU_ERR_UNSUPPORTED;
   const int grid = static_cast<int>(ntiles < st->num_sms ? ntiles : st->num_sms);
-  gemm_bf16_kernel<<<grid, kGemmThreads, GemmCfg::kSmemBytes, stream>>>(ta, tw, p);
-  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  // A programmatic dependent of the previous kernel in the stream: its set-up overlaps that kernel's
+  // tail, and it waits for it (griddepcontrol.wait) before touching global memory.
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = GemmCfg::kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel, ta, tw, p) == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
 // The same product on the two-SM kernel: 256 × 256 tiles, one per cluster of two CTAs.
@@ -389,17 +401,20 @@ hstu_status_t launch_gemm_2sm(DeviceState* st, const void* a, const void* w, voi
   const int clusters = static_cast<int>(ntiles < st->gemm_clusters ? ntiles : st->gemm_clusters);
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // A programmatic dependent of the previous kernel in the stream (as the one-SM launch above).
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(2 * clusters);
   cfg.blockDim = dim3(kGemm2Threads);
   cfg.dynamicSmemBytes = Gemm2Cfg::kSmemBytes;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, gemm_bf16_2sm_kernel, ta, tw, p) == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
