@@ -64,7 +64,8 @@ __host__ __device__ __forceinline__ int item_cost(int pos0, int nrows, int U) {
 constexpr unsigned kErrBadOffsets = 1u;
 constexpr unsigned kErrTimeout = 2u;
 
-constexpr int kSchedThreads = 1024;
+constexpr int kSchedThreads = 256;
+constexpr int kSchedWarps = kSchedThreads / 32;
 constexpr int kMaxCostBins = 4096;
 constexpr int kCachedUsers = 256;  // batches up to this many users keep per-user values in shared memory
 
@@ -105,7 +106,7 @@ __device__ __forceinline__ void block_inclusive_scan2(long long& a, long long& b
   }
   __syncthreads();
   if (warp == 0) {
-    long long wa = scratch[0][lane], wb = scratch[1][lane];
+    long long wa = lane < kSchedWarps ? scratch[0][lane] : 0, wb = lane < kSchedWarps ? scratch[1][lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const long long na = __shfl_up_sync(0xffffffffu, wa, o);
@@ -123,8 +124,8 @@ __device__ __forceinline__ void block_inclusive_scan2(long long& a, long long& b
     a += scratch[0][warp - 1];
     b += scratch[1][warp - 1];
   }
-  total_a = scratch[0][31];
-  total_b = scratch[1][31];
+  total_a = scratch[0][kSchedWarps - 1];
+  total_b = scratch[1][kSchedWarps - 1];
   __syncthreads();
 }
 
@@ -141,7 +142,7 @@ __device__ __forceinline__ long long block_inclusive_scan(long long v, long long
   if (lane == 31) scratch[warp] = v;
   __syncthreads();
   if (warp == 0) {
-    long long w = scratch[lane];
+    long long w = lane < kSchedWarps ? scratch[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       long long n = __shfl_up_sync(0xffffffffu, w, o);
@@ -151,7 +152,7 @@ __device__ __forceinline__ long long block_inclusive_scan(long long v, long long
   }
   __syncthreads();
   if (warp > 0) v += scratch[warp - 1];
-  *total = scratch[31];
+  *total = scratch[kSchedWarps - 1];
   __syncthreads();
   return v;
 }
