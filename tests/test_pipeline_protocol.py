@@ -15,7 +15,8 @@ ahead, for the ring depths the kernel uses (6 slots at d = 128, 10 at d <= 64), 
 constraint kStages <= 2 kSCommits - 2 stated beside the kernel's configuration is the exact limit.
 An event-level model of the group barriers then replays random interleavings of the roles, with
 and without an abort, to show that no arrival ever lands on a phase with no pending arrivals, and
-that the abort path's earlier stand-in arrivals could.
+that the abort path's earlier stand-in arrivals could.  Last, the Q-buffer waits (one buffer at
+d = 128, two at d <= 64) are checked against the MMA warp's per-query-tile commits.
 """
 import numpy as np
 import pytest
@@ -246,3 +247,40 @@ def test_stand_in_arrivals_on_abort_can_meet_a_phase_with_none_pending():
             if "no pending arrivals" in str(e):
                 hit += 1
     assert hit > 0
+
+
+# ---------------------------------------------------------------------------------------------
+# Q buffers.  Query tile s (the s-th the CTA takes) goes into buffer s mod kQBufs.  The MMA warp
+# commits q_empty[b] after a query tile's last score MMA; before loading tile s the producer waits
+# on q_empty[s mod kQBufs] with parity ((s / kQBufs) & 1) ^ 1.  An mbarrier parity wait succeeds once
+# the phase of that parity has completed, and a fresh barrier counts its phase before phase 0 as
+# completed with parity 1.
+# ---------------------------------------------------------------------------------------------
+def q_wait_passes(completions, parity):
+    """try_wait.parity on a barrier that has completed `completions` phases: it passes while the
+    current phase's parity differs from the one asked for, so it cannot tell phases two apart."""
+    return (completions & 1) != parity
+
+
+@pytest.mark.parametrize("qbufs", [1, 2])
+def test_q_buffer_waits_release_exactly_after_the_previous_user_of_the_buffer(qbufs):
+    """For every query tile s, the producer's wait passes exactly when tile s - kQBufs (the buffer's
+    previous user) has committed.  Tiles commit in order, and the producer reached tile s only after
+    its wait for tile s - 1 passed, so tiles up to s - 1 - kQBufs have committed: `done`, the number of
+    committed tiles, is at least s - kQBufs, which keeps the parity wait unambiguous."""
+    for s in range(12):
+        b = s % qbufs
+        parity = ((s // qbufs) & 1) ^ 1
+        for done in range(max(0, s - qbufs), s + 1):
+            completions = sum(1 for t in range(done) if t % qbufs == b)
+            ok = q_wait_passes(completions, parity)
+            assert ok == (s < qbufs or done > s - qbufs), (qbufs, s, done)
+
+
+def test_q_buffer_parity_is_what_catches_a_wrong_buffer_count():
+    """A planted mistake: the parity of two buffers with a single buffer's commits (kQBufs changed in
+    one place only) lets the wait for tile 2 pass before tile 1 has committed."""
+    s, done = 2, 1  # one buffer: tile 2 must wait for tile 1, which has not committed
+    completions = done  # every tile commits on the one barrier
+    parity_two_buffer_formula = ((s // 2) & 1) ^ 1
+    assert q_wait_passes(completions, parity_two_buffer_formula)  # would pass too early
